@@ -1,0 +1,239 @@
+"""Python binding over the C-ABI library ``libfp8nt.so`` (declared in include/fp8_nt.h).
+
+Argument marshalling only: each call checks dtypes, devices and shapes, passes
+raw device pointers, sizes and the current CUDA stream to the library, and
+raises ``Fp8NtError`` on a nonzero status.  Every step of the GEMM runs in the
+library's kernels.  The library is loaded on first use; if it is missing or
+fails to load, the call raises (there is no fallback).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "Fp8NtError",
+    "library_path",
+    "load_library",
+    "gemm_fp8_fp8_bf16_nt",
+    "m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
+    "m_grouped_gemm_fp8_fp8_bf16_nt_masked",
+    "get_m_alignment_for_contiguous_layout",
+    "get_tma_aligned_size",
+    "get_col_major_tma_aligned_tensor",
+    "set_num_sms",
+    "get_num_sms",
+    "get_device_status",
+    "select_config",
+    "force_config",
+    "status_string",
+    "KIND_DENSE",
+    "KIND_CONTIGUOUS",
+    "KIND_MASKED",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libfp8nt.so"
+_lock = threading.Lock()
+_lib = None
+
+KIND_DENSE, KIND_CONTIGUOUS, KIND_MASKED = 0, 1, 2
+
+
+class Fp8NtError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class DgConfig(ctypes.Structure):
+    _fields_ = [("block_m", ctypes.c_int), ("block_n", ctypes.c_int),
+                ("stages", ctypes.c_int), ("sf_stages", ctypes.c_int),
+                ("num_tiles", ctypes.c_int), ("grid", ctypes.c_int),
+                ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load_library():
+    """Load libfp8nt.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with "
+                              "`python -m fp8_fine_grained_nt_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        lib.gemm_fp8_fp8_bf16_nt.argtypes = [P, P, P, P, P, I, I, I, P]
+        lib.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        lib.m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+        lib.get_m_alignment_for_contiguous_layout.argtypes = []
+        lib.get_tma_aligned_size.argtypes = [I, I]
+        lib.set_num_sms.argtypes = [I]
+        lib.get_num_sms.argtypes = []
+        lib.dg_status_string.argtypes = [I]
+        lib.dg_status_string.restype = ctypes.c_char_p
+        lib.dg_get_device_status.argtypes = [P]
+        lib.dg_select_config.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(DgConfig)]
+        lib.dg_force_config.argtypes = [I, I]
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().dg_status_string(status).decode()
+    except ImportError:
+        return "unknown"
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise Fp8NtError(status, where)
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtypes, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+_FP8 = (torch.float8_e4m3fn, torch.uint8)
+_F32 = (torch.float32,)
+
+
+def gemm_fp8_fp8_bf16_nt(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor,
+                         sb: torch.Tensor, d: torch.Tensor, stream=None) -> torch.Tensor:
+    """D[M,N] (bf16) = sum_kb (A_kb B_kb^T) sa[m,kb] sb[n/128,kb].
+
+    a: [M,K] E4M3 (or its uint8 bytes); sa: [ceil(K/128), tma_aligned(M)] fp32
+    column-major LHS scales; b: [N,K] E4M3; sb: [ceil(N/128), ceil(K/128)] fp32;
+    d: [M,N] bf16 output.
+    """
+    M, K = a.shape
+    N = b.shape[0]
+    args = (_dev(a, "a", _FP8, 2), _dev(sa, "sa", _F32, 2), _dev(b, "b", _FP8, 2),
+            _dev(sb, "sb", _F32, 2), _dev(d, "d", (torch.bfloat16,), 2))
+    if tuple(d.shape) != (M, N) or b.shape[1] != K:
+        raise ValueError("shape mismatch between a, b and d")
+    _check(load_library().gemm_fp8_fp8_bf16_nt(*args, M, N, K, _stream_ptr(stream)),
+           "gemm_fp8_fp8_bf16_nt")
+    return d
+
+
+def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(a, sa, b, sb, d, m_indices, stream=None):
+    """Contiguous m-grouped GEMM: row m of A uses expert m_indices[m] (-1 = padding).
+
+    a: [M_sum,K]; sa: [ceil(K/128), M_sum] (M_sum is a multiple of the alignment);
+    b: [G,N,K]; sb: [G, ceil(N/128), ceil(K/128)]; d: [M_sum,N] bf16;
+    m_indices: [M_sum] int32 on the device.
+    """
+    M_sum, K = a.shape
+    G, N = b.shape[0], b.shape[1]
+    args = (_dev(a, "a", _FP8, 2), _dev(sa, "sa", _F32, 2), _dev(b, "b", _FP8, 3),
+            _dev(sb, "sb", _F32, 3), _dev(d, "d", (torch.bfloat16,), 2),
+            _dev(m_indices, "m_indices", (torch.int32,), 1))
+    if tuple(d.shape) != (M_sum, N) or b.shape[2] != K or m_indices.shape[0] != M_sum:
+        raise ValueError("shape mismatch between a, b, d and m_indices")
+    _check(load_library().m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(
+        *args, G, M_sum, N, K, _stream_ptr(stream)), "m_grouped_gemm_fp8_fp8_bf16_nt_contiguous")
+    return d
+
+
+def m_grouped_gemm_fp8_fp8_bf16_nt_masked(a, sa, b, sb, d, masked_m, expected_m: int,
+                                          stream=None):
+    """Masked m-grouped GEMM: group g computes its first masked_m[g] rows only.
+
+    a: [G,M_max,K]; sa: [G, ceil(K/128), tma_aligned(M_max)]; b: [G,N,K];
+    sb: [G, ceil(N/128), ceil(K/128)]; d: [G,M_max,N] bf16; masked_m: [G] int32
+    on the device (never read by the host); expected_m: a host hint for the
+    typical masked_m, used only to choose the tile configuration.
+    """
+    G, M_max, K = a.shape
+    N = b.shape[1]
+    args = (_dev(a, "a", _FP8, 3), _dev(sa, "sa", _F32, 3), _dev(b, "b", _FP8, 3),
+            _dev(sb, "sb", _F32, 3), _dev(d, "d", (torch.bfloat16,), 3),
+            _dev(masked_m, "masked_m", (torch.int32,), 1))
+    if tuple(d.shape) != (G, M_max, N) or tuple(b.shape) != (G, N, K) or masked_m.shape[0] != G:
+        raise ValueError("shape mismatch between a, b, d and masked_m")
+    _check(load_library().m_grouped_gemm_fp8_fp8_bf16_nt_masked(
+        *args, G, M_max, N, K, int(expected_m), _stream_ptr(stream)),
+        "m_grouped_gemm_fp8_fp8_bf16_nt_masked")
+    return d
+
+
+def get_m_alignment_for_contiguous_layout() -> int:
+    return load_library().get_m_alignment_for_contiguous_layout()
+
+
+def get_tma_aligned_size(x: int, element_size: int) -> int:
+    r = load_library().get_tma_aligned_size(int(x), int(element_size))
+    if r < 0:
+        raise Fp8NtError(-r, "get_tma_aligned_size")
+    return r
+
+
+def get_col_major_tma_aligned_tensor(s: torch.Tensor) -> torch.Tensor:
+    """[..., M, nkb] per-row scales -> column-major TMA-aligned [..., nkb, ld] storage.
+
+    A layout helper (torch copy ops, not on the GEMM path): the padding columns
+    between M and ld are left as zeros.
+    """
+    *batch, M, nkb = s.shape
+    ld = get_tma_aligned_size(M, 4)
+    out = torch.zeros((*batch, nkb, ld), dtype=torch.float32, device=s.device)
+    out[..., :M] = s.transpose(-1, -2).float()
+    return out
+
+
+def set_num_sms(n: int) -> None:
+    _check(load_library().set_num_sms(int(n)), "set_num_sms")
+
+
+def get_num_sms() -> int:
+    return load_library().get_num_sms()
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side status word."""
+    return load_library().dg_get_device_status(_stream_ptr(stream))
+
+
+def select_config(kind: int, M: int, N: int, K: int, num_groups: int = 1,
+                  expected_m: int = 0, num_sms: int = 148) -> dict:
+    """The tile configuration the library would launch (host logic only, no GPU)."""
+    cfg = DgConfig()
+    _check(load_library().dg_select_config(kind, M, N, K, num_groups, expected_m, num_sms,
+                                           ctypes.byref(cfg)), "dg_select_config")
+    return cfg.as_dict()
+
+
+def force_config(block_m: int = 0, block_n: int = 0) -> None:
+    """Pin the tile shape for later calls (0, 0 = automatic).  For tests."""
+    _check(load_library().dg_force_config(int(block_m), int(block_n)), "dg_force_config")
