@@ -1,0 +1,513 @@
+// C-ABI entry points of libfp8nt.so (declared in include/fp8_nt.h): argument
+// validation, tile-configuration choice, TMA descriptor encoding and launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <math.h>
+#include <mutex>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "../../include/fp8_nt.h"
+#include "launch.h"
+#include "params.h"
+
+using namespace fp8nt;
+
+namespace {
+
+// ------------------------------------------------------------------ kernels
+
+struct Candidate {
+    int mw;
+    int bn;
+    LaunchFn launch;
+};
+
+const Candidate kCandidates[] = {
+#define FP8NT_KERNEL(mw, bn) {mw, bn, launch_mw##mw##_bn##bn},
+#include "kernels.def"
+#undef FP8NT_KERNEL
+};
+constexpr int kNumCandidates = sizeof(kCandidates) / sizeof(kCandidates[0]);
+
+constexpr int kDefaultSms = 148;           // B200
+constexpr int kDefaultMaxSmem = 232448;    // 227 KB opt-in per block on sm_100
+constexpr int kMaxStages = 12;
+constexpr int kMinStages = 2;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull; // 2 s per pipeline wait
+
+// ------------------------------------------------------------------ devices
+
+// The device status word.  Host code must not take this symbol's address
+// directly: its device address is fetched per device with
+// cudaGetSymbolAddress and passed to the kernels.
+__device__ unsigned int g_status_word;
+
+struct DeviceInfo {
+    bool ready;
+    int sm_count;
+    int cc_major;
+    int cc_minor;
+    int max_smem;
+    unsigned int *status;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+int g_num_sms_limit = 0;
+int g_forced_bm = 0, g_forced_bn = 0;
+uint64_t g_timeout_ns = 0;
+
+int device_info(DeviceInfo **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_devices[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess)
+            return DG_ERR_CUDA;
+        if (d.cc_major != 10 || d.cc_minor != 0)
+            return DG_ERR_UNSUPPORTED_ARCH;
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess)
+            return DG_ERR_CUDA;
+        d.status = static_cast<unsigned int *>(addr);
+        d.ready = true;
+    }
+    *out = &d;
+    return DG_OK;
+}
+
+uint64_t wait_timeout_ns()
+{
+    if (g_timeout_ns == 0) {
+        const char *env = getenv("DG_WAIT_TIMEOUT_MS");
+        long ms = env ? atol(env) : 0;
+        g_timeout_ns = ms > 0 ? (uint64_t)ms * 1000000ull : kDefaultTimeoutNs;
+    }
+    return g_timeout_ns;
+}
+
+// ------------------------------------------------------------------ TMA
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `elem` bytes per element, row pitch
+// `pitch_elems`, box [box_rows][box_cols].
+int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType type, int elem,
+                 uint64_t cols, uint64_t rows, uint64_t pitch_elems, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle swizzle)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return DG_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch_elems * (uint64_t)elem};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ config
+
+int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
+
+struct Problem {
+    int kind;
+    int M;          // dense M / contiguous M_sum / masked M_max
+    int N;
+    int K;
+    int groups;
+    int expected_m; // masked only
+};
+
+// Rough cycle estimate of a (MW, BN) choice on `sms` SMs: whole waves of
+// tiles, each tile nkb K blocks long, a K block limited by the tensor pipe
+// (2 * BN cycles per 128-row MMA group at 8192 FP8 MAC/clk), operand delivery
+// (~64 B/clk/SM from L2) or the promotion FMAs (BN cycles per 128 rows).
+double estimate_cycles(const Problem &pb, int mw, int bn, int sms, int *tiles_out)
+{
+    const int bm = 128 * mw;
+    const int nkb = pb.K / 128;
+    long m_blocks;
+    int rows_eff;
+    if (pb.kind == DG_KIND_MASKED) {
+        int em = pb.expected_m > 0 ? pb.expected_m : pb.M;
+        em = em > pb.M ? pb.M : em;
+        em = em < 1 ? 1 : em;
+        m_blocks = (long)pb.groups * ceil_div(em, bm);
+        rows_eff = em < bm ? em : bm;
+    } else {
+        m_blocks = ceil_div(pb.M, bm);
+        rows_eff = pb.M < bm ? pb.M : bm;
+    }
+    const long n_blocks = ceil_div(pb.N, bn);
+    const long tiles = m_blocks * n_blocks;
+    const long waves = (tiles + sms - 1) / sms;
+    const int halves = (mw == 2 && rows_eff > 128) ? 2 : 1;
+    const double mma = 2.0 * bn * halves;
+    const double l2 = (double)(rows_eff + bn) * 128.0 / 64.0;
+    const double epi = (double)bn * halves;
+    double per_kb = mma > l2 ? mma : l2;
+    per_kb = per_kb > epi ? per_kb : epi;
+    per_kb += 40.0;
+    const double tile = nkb * per_kb + 1000.0;
+    if (tiles_out)
+        *tiles_out = (int)(tiles > 0x7fffffff ? 0x7fffffff : tiles);
+    return waves * tile;
+}
+
+int plan_for(const Problem &pb, int mw, int bn, int max_smem, int *stages, int *sf_stages,
+             SmemPlan *plan)
+{
+    const int nkb = pb.K / 128;
+    const int prefix_ints = pb.kind == DG_KIND_MASKED ? 2 * pb.groups + 1 : 0;
+    for (int s = kMaxStages; s >= kMinStages; --s) {
+        const int sf = s + 4;
+        SmemPlan p = make_smem_plan(mw, bn, s, sf, nkb, prefix_ints);
+        if ((int)p.total + 1024 <= max_smem) {
+            *stages = s;
+            *sf_stages = sf;
+            *plan = p;
+            return DG_OK;
+        }
+    }
+    return DG_ERR_UNSUPPORTED_SHAPE;
+}
+
+int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand, dg_config *cfg,
+           SmemPlan *plan)
+{
+    const Candidate *best = nullptr;
+    double best_cost = 0;
+    for (int i = 0; i < kNumCandidates; ++i) {
+        const Candidate &c = kCandidates[i];
+        if (g_forced_bm && (c.mw * 128 != g_forced_bm || c.bn != g_forced_bn))
+            continue;
+        if (pb.kind == DG_KIND_CONTIGUOUS && c.mw != 1)
+            continue; // a 256-row tile could straddle two 128-aligned experts
+        int st, sf;
+        SmemPlan p;
+        if (plan_for(pb, c.mw, c.bn, max_smem, &st, &sf, &p) != DG_OK)
+            continue;
+        const double cost = estimate_cycles(pb, c.mw, c.bn, sms, nullptr);
+        // ties: wider tile first (fewer re-reads of A), then one M half
+        const bool better = !best || cost < best_cost * (1 - 1e-9) ||
+                            (fabs(cost - best_cost) <= best_cost * 1e-9 &&
+                             (c.bn > best->bn || (c.bn == best->bn && c.mw < best->mw)));
+        if (better) {
+            best = &c;
+            best_cost = cost;
+        }
+    }
+    if (!best)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    int st, sf;
+    plan_for(pb, best->mw, best->bn, max_smem, &st, &sf, plan);
+    const int bm = best->mw * 128;
+    long tiles;
+    if (pb.kind == DG_KIND_MASKED)
+        tiles = (long)pb.groups * ceil_div(pb.M, bm) * ceil_div(pb.N, best->bn);
+    else
+        tiles = (long)ceil_div(pb.M, bm) * ceil_div(pb.N, best->bn);
+    if (tiles > 0x7fffffffL)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    cfg->block_m = bm;
+    cfg->block_n = best->bn;
+    cfg->stages = st;
+    cfg->sf_stages = sf;
+    cfg->num_tiles = (int)tiles;
+    cfg->grid = (int)(tiles < sms ? tiles : sms);
+    if (cfg->grid < 1)
+        cfg->grid = 1;
+    cfg->smem_bytes = (int)plan->total + 1024;
+    const int need = 2 * best->mw * best->bn;
+    cfg->tmem_cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
+    *out_cand = best;
+    return DG_OK;
+}
+
+int effective_sms(const DeviceInfo *d)
+{
+    int n = d ? d->sm_count : kDefaultSms;
+    if (g_num_sms_limit > 0 && g_num_sms_limit < n)
+        n = g_num_sms_limit;
+    return n;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(const void *A, const float *sa, const void *B, const float *sb, void *D, int M,
+                 int N, int K)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (K == 0 || K % 128 != 0 || N % 8 != 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0)
+        return DG_OK;
+    if (!A || !sa || !B || !sb || !D)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(A) || !aligned16(sa) || !aligned16(B) || !aligned16(sb) || !aligned16(D))
+        return DG_ERR_MISALIGNED;
+    return DG_OK;
+}
+
+// Shared launch path for the three forms.
+int run(const Problem &pb, const void *A, const float *sa, const void *B, const float *sb, void *D,
+        const int *m_indices, const int *masked_m, cudaStream_t stream)
+{
+    DeviceInfo *dev = nullptr;
+    int st = device_info(&dev);
+    if (st != DG_OK)
+        return st;
+    const int sms = effective_sms(dev);
+    const Candidate *cand = nullptr;
+    dg_config cfg;
+    SmemPlan plan;
+    st = choose(pb, sms, dev->max_smem, &cand, &cfg, &plan);
+    if (st != DG_OK)
+        return st;
+
+    const int nkb = pb.K / 128;
+    const int nnb = ceil_div(pb.N, 128);
+    const int groups = pb.kind == DG_KIND_DENSE ? 1 : pb.groups;
+    const int ld_sa = get_tma_aligned_size(pb.M, 4);
+
+    CUtensorMap tmap_a, tmap_b, tmap_sa;
+    const long a_rows = pb.kind == DG_KIND_MASKED ? (long)groups * pb.M : pb.M;
+    const long b_rows = (long)groups * pb.N;
+    const long sa_rows = pb.kind == DG_KIND_MASKED ? (long)groups * nkb : nkb;
+    if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, a_rows, pb.K, 128,
+                           128, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+        return st;
+    if ((st = make_tmap_2d(&tmap_b, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, b_rows, pb.K, 128,
+                           cfg.block_n, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+        return st;
+    if ((st = make_tmap_2d(&tmap_sa, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ld_sa, sa_rows, ld_sa,
+                           128, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+        return st;
+
+    Params p;
+    memset(&p, 0, sizeof(p));
+    p.kind = pb.kind;
+    p.M = pb.M;
+    p.N = pb.N;
+    p.K = pb.K;
+    p.num_groups = groups;
+    p.nkb = nkb;
+    p.nnb = nnb;
+    p.m_blocks = ceil_div(pb.M, cfg.block_m);
+    p.n_blocks = ceil_div(pb.N, cfg.block_n);
+    p.num_tiles = cfg.num_tiles;
+    p.stages = cfg.stages;
+    p.sf_stages = cfg.sf_stages;
+    p.plan = plan;
+    p.sb = sb;
+    p.m_indices = m_indices;
+    p.masked_m = masked_m;
+    p.D = static_cast<uint16_t *>(D);
+    p.status = dev->status;
+    p.timeout_ns = wait_timeout_ns();
+
+    LaunchArgs args;
+    args.tmap_a = &tmap_a;
+    args.tmap_b = &tmap_b;
+    args.tmap_sa = &tmap_sa;
+    args.params = &p;
+    args.grid = cfg.grid;
+    args.smem_bytes = cfg.smem_bytes;
+    args.stream = stream;
+    return cand->launch(args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+} // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+int gemm_fp8_fp8_bf16_nt(const void *A, const float *sa, const void *B, const float *sb, void *D,
+                         int M, int N, int K, dg_stream_t stream)
+{
+    int st = check_common(A, sa, B, sb, D, M, N, K);
+    if (st != DG_OK || M == 0 || N == 0)
+        return st;
+    Problem pb{DG_KIND_DENSE, M, N, K, 1, 0};
+    return run(pb, A, sa, B, sb, D, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *A, const float *sa, const void *B,
+                                              const float *sb, void *D, const int *m_indices,
+                                              int num_groups, int M_sum, int N, int K,
+                                              dg_stream_t stream)
+{
+    if (num_groups <= 0)
+        return DG_ERR_INVALID_ARGUMENT;
+    int st = check_common(A, sa, B, sb, D, M_sum, N, K);
+    if (st != DG_OK || M_sum == 0 || N == 0)
+        return st;
+    if (!m_indices)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(m_indices))
+        return DG_ERR_MISALIGNED;
+    if (M_sum % get_m_alignment_for_contiguous_layout() != 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    if ((long)num_groups * N > 0x7fffffffL)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    Problem pb{DG_KIND_CONTIGUOUS, M_sum, N, K, num_groups, 0};
+    return run(pb, A, sa, B, sb, D, m_indices, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *A, const float *sa, const void *B,
+                                          const float *sb, void *D, const int *masked_m, int G,
+                                          int M_max, int N, int K, int expected_m,
+                                          dg_stream_t stream)
+{
+    if (G <= 0 || expected_m < 0)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (G > MAX_MASKED_GROUPS)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    int st = check_common(A, sa, B, sb, D, M_max, N, K);
+    if (st != DG_OK || M_max == 0 || N == 0)
+        return st;
+    if (!masked_m)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(masked_m))
+        return DG_ERR_MISALIGNED;
+    if ((long)G * M_max > 0x7fffffffL || (long)G * N > 0x7fffffffL)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    Problem pb{DG_KIND_MASKED, M_max, N, K, G, expected_m};
+    return run(pb, A, sa, B, sb, D, nullptr, masked_m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int get_m_alignment_for_contiguous_layout(void) { return 128; }
+
+int get_tma_aligned_size(int x, int element_size)
+{
+    if (x < 0 || element_size <= 0 || 16 % element_size != 0)
+        return -DG_ERR_INVALID_ARGUMENT;
+    const int align = 16 / element_size;
+    return (x + align - 1) / align * align;
+}
+
+int set_num_sms(int n)
+{
+    g_num_sms_limit = n > 0 ? n : 0;
+    return DG_OK;
+}
+
+int get_num_sms(void)
+{
+    int count = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+        if (g_num_sms_limit > 0 && g_num_sms_limit < count)
+            return g_num_sms_limit;
+        return count;
+    }
+    cudaGetLastError(); // no device: clear the sticky-free error state
+    return g_num_sms_limit;
+}
+
+const char *dg_status_string(int status)
+{
+    switch (status) {
+    case DG_OK: return "ok";
+    case DG_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case DG_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case DG_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DG_ERR_UNSUPPORTED_ARCH: return "current device is not sm_100 (B200)";
+    case DG_ERR_CUDA: return "CUDA call failed";
+    case DG_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case DG_ERR_DEVICE_BAD_INDEX: return "masked_m or m_indices out of range";
+    default: return "unknown status";
+    }
+}
+
+int dg_get_device_status(dg_stream_t stream)
+{
+    DeviceInfo *dev = nullptr;
+    int st = device_info(&dev);
+    if (st != DG_OK)
+        return st;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DG_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, dev->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return DG_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return DG_ERR_CUDA;
+    }
+    if (word & DEVERR_TIMEOUT)
+        return DG_ERR_DEVICE_TIMEOUT;
+    if (word & DEVERR_BAD_INDEX)
+        return DG_ERR_DEVICE_BAD_INDEX;
+    return DG_OK;
+}
+
+int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected_m, int num_sms,
+                     dg_config *out)
+{
+    if (!out || kind < 0 || kind > 2 || M <= 0 || N <= 0 || K <= 0 || num_groups <= 0)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (K % 128 != 0 || N % 8 != 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    if (kind == DG_KIND_MASKED && num_groups > MAX_MASKED_GROUPS)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    int sms = num_sms > 0 ? num_sms : (g_num_sms_limit > 0 ? g_num_sms_limit : kDefaultSms);
+    Problem pb{kind, M, N, K, kind == DG_KIND_DENSE ? 1 : num_groups, expected_m};
+    const Candidate *cand = nullptr;
+    SmemPlan plan;
+    return choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);
+}
+
+int dg_force_config(int block_m, int block_n)
+{
+    if (block_m == 0 && block_n == 0) {
+        g_forced_bm = g_forced_bn = 0;
+        return DG_OK;
+    }
+    for (int i = 0; i < kNumCandidates; ++i)
+        if (kCandidates[i].mw * 128 == block_m && kCandidates[i].bn == block_n) {
+            g_forced_bm = block_m;
+            g_forced_bn = block_n;
+            return DG_OK;
+        }
+    return DG_ERR_UNSUPPORTED_SHAPE;
+}
+
+} // extern "C"

@@ -1,0 +1,28 @@
+// Host-side launch interface between the C-ABI layer and the kernel
+// instantiations (one launcher per tile shape listed in kernels.def).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "params.h"
+
+namespace fp8nt {
+
+struct LaunchArgs {
+    const CUtensorMap *tmap_a;
+    const CUtensorMap *tmap_b;
+    const CUtensorMap *tmap_sa;
+    const Params *params;
+    int grid;
+    int smem_bytes;
+    cudaStream_t stream;
+};
+
+typedef cudaError_t (*LaunchFn)(const LaunchArgs &);
+
+#define FP8NT_KERNEL(mw, bn) cudaError_t launch_mw##mw##_bn##bn(const LaunchArgs &);
+#include "kernels.def"
+#undef FP8NT_KERNEL
+
+} // namespace fp8nt

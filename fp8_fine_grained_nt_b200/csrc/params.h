@@ -1,0 +1,97 @@
+// Kernel parameters and the shared-memory plan, shared by the host launcher
+// and the kernel.
+#pragma once
+
+#include <stdint.h>
+
+namespace fp8nt {
+
+enum GemmKind : int { KIND_DENSE = 0, KIND_CONTIGUOUS = 1, KIND_MASKED = 2 };
+
+constexpr int BLOCK_K = 128;          // one scale block of K = one 128-byte swizzle row
+constexpr int HALF_M = 128;           // rows of one tcgen05 MMA (cta_group::1, M = 128)
+constexpr int MMA_K = 32;             // K of one kind::f8f6f4 MMA
+constexpr int NUM_THREADS = 384;      // 3 warpgroups
+constexpr int FIRST_EPI_WARP = 4;     // warps 4..11 run the promotion epilogue
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int MAX_SB_BLOCKS = 3;      // a BLOCK_N <= 256 tile spans at most 3 sb blocks
+constexpr int MAX_MASKED_GROUPS = 1024;
+constexpr int REGS_PRODUCER = 56;     // per-thread registers after setmaxnreg
+constexpr int REGS_EPILOGUE = 224;
+constexpr int REGS_AT_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
+
+static_assert(4 * 32 * REGS_PRODUCER + 8 * 32 * REGS_EPILOGUE <= NUM_THREADS * REGS_AT_LAUNCH,
+              "register split exceeds the launch allocation");
+
+// Device status bits (read back by dg_get_device_status).
+constexpr uint32_t DEVERR_TIMEOUT = 1u;
+constexpr uint32_t DEVERR_BAD_INDEX = 2u;
+
+struct SmemPlan {
+    uint32_t stage_bytes;   // A (MW x 16 KB) + B (BN x 128 B)
+    uint32_t a_bytes;
+    uint32_t off_stages;    // 1024-aligned
+    uint32_t off_sf;        // LHS-scale ring: sf_stages x MW x 128 floats
+    uint32_t sf_slot_bytes;
+    uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
+    uint32_t sb_pitch;      // floats per sb row in smem (nkb rounded up to 4)
+    uint32_t off_prefix;    // masked: (G + 1) ints of per-group tile prefix sums
+    uint32_t off_bars;      // all mbarriers
+    uint32_t off_misc;      // tmem base address, abort flag
+    uint32_t total;         // bytes, excluding the 1024 B alignment slack
+};
+
+struct Params {
+    int kind;
+    int M;          // dense: M; contiguous: M_sum; masked: M_max
+    int N;
+    int K;
+    int num_groups; // 1 for dense
+    int nkb;        // K / 128
+    int nnb;        // ceil(N / 128)
+    int m_blocks;   // dense / contiguous: ceil(M / BLOCK_M); masked: per-group maximum
+    int n_blocks;   // ceil(N / BLOCK_N)
+    int num_tiles;  // dense / contiguous; masked tiles are counted on the device
+    int stages;
+    int sf_stages;
+    SmemPlan plan;
+    const float *sb;
+    const int *m_indices;
+    const int *masked_m;
+    uint16_t *D;    // BF16 bits
+    unsigned int *status; // device status word (DEVERR_* bits)
+    uint64_t timeout_ns;  // limit on any single pipeline wait
+};
+
+__host__ __device__ inline uint32_t align_up_u32(uint32_t x, uint32_t a)
+{
+    return (x + a - 1) / a * a;
+}
+
+// Shared-memory layout for a (MW, BN) kernel with the given ring depths.
+__host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, int sf_stages,
+                                                   int nkb, int prefix_ints)
+{
+    SmemPlan p;
+    p.a_bytes = (uint32_t)mw * HALF_M * BLOCK_K;
+    p.stage_bytes = p.a_bytes + (uint32_t)bn * BLOCK_K;
+    p.off_stages = 0;
+    uint32_t off = p.stage_bytes * (uint32_t)stages;
+    p.off_sf = align_up_u32(off, 128);
+    p.sf_slot_bytes = (uint32_t)mw * HALF_M * 4;
+    off = p.off_sf + p.sf_slot_bytes * (uint32_t)sf_stages;
+    p.sb_pitch = align_up_u32((uint32_t)nkb, 4);
+    p.off_sb = align_up_u32(off, 128);
+    off = p.off_sb + 2u * MAX_SB_BLOCKS * p.sb_pitch * 4u;
+    p.off_prefix = align_up_u32(off, 16);
+    off = p.off_prefix + 4u * (uint32_t)prefix_ints;
+    p.off_bars = align_up_u32(off, 8);
+    // full/empty per stage, full/empty per sf stage, tmem full/empty x2,
+    // sb full/empty x2, one "all MMAs done" barrier
+    off = p.off_bars + 8u * (2u * stages + 2u * sf_stages + 4u + 4u + 1u);
+    p.off_misc = align_up_u32(off, 16);
+    p.total = p.off_misc + 16;
+    return p;
+}
+
+} // namespace fp8nt

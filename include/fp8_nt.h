@@ -1,0 +1,165 @@
+/*
+ * fp8_nt.h — C ABI of libfp8nt.so: FP8 (E4M3) NT GEMM with fine-grained
+ * scaling and BF16 output, for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (DeepGEMM README, introduction: FP8 GEMMs "with
+ * fine-grained scaling" as proposed in DeepSeek-V3; usage: NT format only):
+ *
+ *   D[m,n] = sum over 128-wide K blocks kb of
+ *              ( sum_{k in kb} A[m,k] * B[n,k] ) * sa[m,kb] * sb[n/128,kb]
+ *
+ * accumulated in FP32 (each K block's tensor-core partial is promoted into an
+ * FP32 accumulator with its scale product: the README's two-level
+ * accumulation) and rounded to BF16 (round-to-nearest-even) on store.
+ *
+ * Common conventions for the three GEMM entry points
+ * ---------------------------------------------------
+ * Pointers.  Every pointer is CUDA device memory owned by the caller.  The
+ *   library never allocates, frees or keeps a reference to it after the call
+ *   returns; it reads A, sa, B, sb (and m_indices / masked_m) and writes D.
+ *   Every pointer must be 16-byte aligned.
+ * Element types.  A and B hold E4M3 bytes (1 sign, 4 exponent bits with bias
+ *   7, 3 mantissa bits; 0x7F/0xFF are NaN).  sa and sb are IEEE FP32.  D is
+ *   BF16 (stored as uint16).
+ * Layouts.  "NT": A is [M,K] row-major (K contiguous) and B is [N,K] row-major
+ *   (K contiguous) (DeepGEMM README, usage).  sa is COLUMN-MAJOR and
+ *   TMA-aligned: sa[kb * ld + m] with ld = get_tma_aligned_size(M, 4)
+ *   (README, utility functions: get_tma_aligned_size,
+ *   get_col_major_tma_aligned_tensor).  sb is row-major [ceil(N/128)][K/128].
+ *   D is row-major [M,N] BF16.
+ * Shape rules.  K % 128 == 0 (the scale block), N % 8 == 0 (16-byte rows of
+ *   D), M >= 0.  A call with M == 0 (or all groups empty) does nothing.
+ * Stream.  Work is enqueued on `stream` (a cudaStream_t / CUstream; NULL = the
+ *   legacy default stream) and runs asynchronously.  No call synchronises,
+ *   allocates or reads device memory on the host, so every call can be
+ *   captured in a CUDA graph.
+ * Errors.  Arguments the host can check are checked before anything is
+ *   launched; the call then returns a nonzero dg_status and enqueues nothing.
+ *   Errors the host cannot see (a masked_m or m_indices value out of range, a
+ *   pipeline wait that timed out) are recorded in a device status word,
+ *   read and cleared by dg_get_device_status().  The kernel never traps.
+ */
+#ifndef FP8_NT_H
+#define FP8_NT_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dg_stream_t; /* same type as cudaStream_t */
+
+typedef enum dg_status {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARGUMENT = 1,  /* null pointer, negative size, bad count */
+    DG_ERR_MISALIGNED = 2,        /* a pointer not 16-byte aligned */
+    DG_ERR_UNSUPPORTED_SHAPE = 3, /* K % 128, N % 8, or a size over a limit */
+    DG_ERR_UNSUPPORTED_ARCH = 4,  /* current device is not sm_100 */
+    DG_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed */
+    DG_ERR_DEVICE_TIMEOUT = 6,    /* device: a pipeline wait ran out (kernel exited early) */
+    DG_ERR_DEVICE_BAD_INDEX = 7   /* device: masked_m / m_indices out of range */
+} dg_status;
+
+/* Dense GEMM (DeepGEMM README, usage: deep_gemm.gemm_fp8_fp8_bf16_nt, the
+ * basic non-grouped FP8 GEMM).
+ *   A  [M,K] E4M3          sa [K/128][get_tma_aligned_size(M,4)] FP32
+ *   B  [N,K] E4M3          sb [ceil(N/128)][K/128] FP32
+ *   D  [M,N] BF16 (written in full) */
+int gemm_fp8_fp8_bf16_nt(const void *A, const float *sa, const void *B, const float *sb,
+                         void *D, int M, int N, int K, dg_stream_t stream);
+
+/* Contiguous m-grouped GEMM (DeepGEMM README, grouped GEMMs: tokens of all
+ * experts concatenated into one tensor, each expert segment aligned to
+ * get_m_alignment_for_contiguous_layout(); only the M axis is grouped, all
+ * experts share N and K).
+ *   A  [M_sum,K] E4M3       sa [K/128][M_sum] FP32 (M_sum is a multiple of the
+ *                                                  alignment, so ld = M_sum)
+ *   B  [num_groups,N,K]     sb [num_groups][ceil(N/128)][K/128]
+ *   D  [M_sum,N] BF16
+ *   m_indices [M_sum] int32 on the device: the expert of each row, or -1 on a
+ *   padding row.  Each aligned block of rows takes the expert of its first
+ *   row; all non-padding rows of a block must share it.  Rows marked -1 are
+ *   not written; a block whose first row is -1 is skipped.  An expert index
+ *   >= num_groups sets DG_ERR_DEVICE_BAD_INDEX and its block is skipped.
+ *   M_sum % get_m_alignment_for_contiguous_layout() must be 0. */
+int m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *A, const float *sa, const void *B,
+                                              const float *sb, void *D, const int *m_indices,
+                                              int num_groups, int M_sum, int N, int K,
+                                              dg_stream_t stream);
+
+/* Masked m-grouped GEMM (DeepGEMM README, grouped GEMMs: for CUDA-graph
+ * decode, when the host does not know how many tokens each expert got; the
+ * kernel computes only the valid part given by a mask tensor).
+ *   A  [G,M_max,K] E4M3      sa [G][K/128][get_tma_aligned_size(M_max,4)]
+ *   B  [G,N,K]               sb [G][ceil(N/128)][K/128]
+ *   D  [G,M_max,N] BF16
+ *   masked_m [G] int32 on the device: rows 0..masked_m[g]-1 of group g are
+ *   computed; rows at or beyond masked_m[g] are never written.  The host never
+ *   reads masked_m.  A value outside [0, M_max] sets DG_ERR_DEVICE_BAD_INDEX
+ *   and is clamped into range.
+ *   expected_m: the caller's estimate of a typical masked_m (a hint for the
+ *   tile choice only; 0 = assume M_max). */
+int m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *A, const float *sa, const void *B,
+                                          const float *sb, void *D, const int *masked_m, int G,
+                                          int M_max, int N, int K, int expected_m,
+                                          dg_stream_t stream);
+
+/* Row alignment of each expert segment in the contiguous layout (DeepGEMM
+ * README, utility functions: get_m_alignment_for_contiguous_layout).  128. */
+int get_m_alignment_for_contiguous_layout(void);
+
+/* Smallest count >= x whose size in bytes (x * element_size) is a multiple of
+ * 16: the TMA-aligned leading dimension (DeepGEMM README, utility functions:
+ * get_tma_aligned_size).  element_size must divide 16; returns
+ * -DG_ERR_INVALID_ARGUMENT otherwise or if x < 0. */
+int get_tma_aligned_size(int x, int element_size);
+
+/* Upper bound on the SMs the kernels use (DeepGEMM README, utility
+ * functions: set_num_sms / get_num_sms).  n <= 0 restores "all SMs of the
+ * current device".  Returns DG_OK.  get_num_sms() returns the bound in force
+ * (the device's SM count when unset and a device is present, else 0). */
+int set_num_sms(int n);
+int get_num_sms(void);
+
+/* Static description of a dg_status value. */
+const char *dg_status_string(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * (DG_OK, DG_ERR_DEVICE_TIMEOUT or DG_ERR_DEVICE_BAD_INDEX), or DG_ERR_CUDA if
+ * the synchronisation itself failed. */
+int dg_get_device_status(dg_stream_t stream);
+
+/* Tile configuration chosen for a call (host logic; no GPU needed). */
+typedef struct dg_config {
+    int block_m;    /* rows per CTA tile: 128 or 256 (two 128-row MMAs) */
+    int block_n;    /* columns per CTA tile: a multiple of 16 in [16, 256] */
+    int stages;     /* depth of the shared-memory operand ring */
+    int sf_stages;  /* depth of the LHS-scale ring */
+    int num_tiles;  /* tiles to compute (upper bound for the masked form) */
+    int grid;       /* persistent CTAs launched */
+    int smem_bytes; /* dynamic shared memory per CTA */
+    int tmem_cols;  /* tensor-memory columns allocated per CTA */
+} dg_config;
+
+enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2 };
+
+/* The configuration a call of `kind` would use.  For DG_KIND_DENSE: M, N, K;
+ * for DG_KIND_CONTIGUOUS: M = M_sum; for DG_KIND_MASKED: M = M_max and
+ * expected_m as in the masked call.  num_sms <= 0 means the bound from
+ * set_num_sms, else 148.  The selection is deterministic (DeepGEMM README, JIT
+ * design: block sizes and pipeline stages chosen without auto-tuning) and
+ * favours tile counts that fill the SMs, with non-power-of-two BLOCK_N where
+ * that helps (README, unaligned block sizes).  Returns DG_OK or an argument
+ * error. */
+int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected_m,
+                     int num_sms, dg_config *out);
+
+/* Test hook: pin block_m / block_n for later calls (0, 0 restores automatic
+ * choice).  Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is
+ * built. */
+int dg_force_config(int block_m, int block_n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8_NT_H */

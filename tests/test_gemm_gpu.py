@@ -1,0 +1,258 @@
+"""GPU parity: the CUDA path (through the Python binding and the C ABI) against
+the CPU oracle on the same seeded inputs.
+
+Small cases compare every element; full-size cases (the measured workloads, in
+the configuration the benchmark launches) compare sampled elements and whole
+rows, and check the properties that hold at any size: rows that must stay
+untouched keep their sentinel bits, and repeated calls are bit-identical.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_fine_grained_nt_b200 as fp8
+from fp8_fine_grained_nt_b200 import inputs
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+BUILT_SHAPES = None
+
+
+def built_shapes():
+    from fp8_fine_grained_nt_b200 import build
+    return build.kernel_shapes()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fp8_fine_grained_nt_b200 import build
+    build.build()
+    fp8.force_config(0, 0)
+    yield
+    fp8.force_config(0, 0)
+
+
+def check_status():
+    st = fp8.get_device_status()
+    assert st == 0, f"device status {st}: {fp8.status_string(st)}"
+
+
+# --------------------------------------------------------------------- dense
+
+
+@pytest.mark.parametrize("mw,bn", built_shapes())
+def test_dense_every_kernel_shape_ragged(mw, bn):
+    """Each built tile shape on a shape with ragged M, N tails and several K blocks."""
+    prob = inputs.make_dense(300, 400, 512, seed=100 + bn + mw)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
+    fp8.force_config(128 * mw, bn)
+    try:
+        d = H.run_dense(prob)
+    finally:
+        fp8.force_config(0, 0)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense mw{mw} bn{bn}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 128), (1, 16, 128), (5, 24, 256), (128, 128, 512),
+                                   (129, 136, 384), (257, 8, 128), (64, 2112, 7168)])
+def test_dense_auto_config(M, N, K):
+    prob = inputs.make_dense(M, N, K, seed=M * 7 + N + K)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, M, N, K)
+    d = H.run_dense(prob)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense {M}x{N}x{K}")
+
+
+def test_dense_exact_small_integers():
+    """Unit scales and small-integer FP8 values give an exact result: bit-exact BF16."""
+    M, N, K = 200, 144, 512
+    one = torch.tensor([1.0]).to(torch.float8_e4m3fn).view(torch.uint8)
+    vals = torch.tensor([float(i % 4 + 1) for i in range(M)]).to(torch.float8_e4m3fn)
+    a = vals.view(torch.uint8)[:, None].expand(M, K).contiguous()
+    b = one.expand(N, K).contiguous()
+    ld = inputs.tma_aligned_size(M, 4)
+    prob = inputs.DenseProblem(M, N, K, a, torch.ones(K // 128, ld), b,
+                               torch.ones(math.ceil(N / 128), K // 128))
+    d = H.run_dense(prob)
+    got = H.bf16_bits_to_f64(d)
+    expect = np.array([[512.0 * (i % 4 + 1)] * N for i in range(M)])
+    assert np.array_equal(got, expect)
+
+
+def test_dense_deterministic_and_no_stray_writes():
+    prob = inputs.make_dense(250, 264, 1024, seed=5)
+    d1 = H.run_dense(prob)
+    d2 = H.run_dense(prob)
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+    # a larger buffer: only the M x N region may change
+    big = H.sentinel_like((prob.M + 3, prob.N))
+    H.run_dense(prob, big[: prob.M])
+    assert H.untouched(big[prob.M:]).all()
+
+
+# --------------------------------------------------------------------- contiguous
+
+
+def test_contiguous_small_all_rows():
+    prob = inputs.make_contiguous(4, 272, 384, seed=21, counts=[0, 5, 130, 257])
+    ref = oracle.gemm_contiguous(prob.a, prob.sa, prob.b, prob.sb, prob.m_indices,
+                                 prob.num_groups, prob.M_sum, prob.N, prob.K)
+    d = H.run_contiguous(prob)
+    check_status()
+    valid = prob.m_indices.numpy() >= 0
+    H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], "contiguous small")
+    assert H.untouched(d)[~valid].all(), "padding rows were written"
+
+
+@pytest.mark.parametrize("bn", [64, 112, 256])
+def test_contiguous_forced_shapes(bn):
+    prob = inputs.make_contiguous(3, 320, 256, seed=22 + bn, counts=[129, 1, 300])
+    ref = oracle.gemm_contiguous(prob.a, prob.sa, prob.b, prob.sb, prob.m_indices,
+                                 prob.num_groups, prob.M_sum, prob.N, prob.K)
+    fp8.force_config(128, bn)
+    try:
+        d = H.run_contiguous(prob)
+    finally:
+        fp8.force_config(0, 0)
+    check_status()
+    valid = prob.m_indices.numpy() >= 0
+    H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], f"contiguous bn{bn}")
+    assert H.untouched(d)[~valid].all()
+
+
+def test_contiguous_bad_expert_index_reported():
+    prob = inputs.make_contiguous(2, 64, 128, seed=23, counts=[128, 128])
+    prob.m_indices[128:256] = 7  # out of range for 2 experts
+    d = H.run_contiguous(prob)
+    assert fp8.get_device_status() == 7
+    assert H.untouched(d)[128:].all()
+    assert fp8.get_device_status() == 0  # cleared
+
+
+# --------------------------------------------------------------------- masked
+
+
+@pytest.mark.parametrize("expected_m", [0, 1, 100])
+def test_masked_small_all_rows(expected_m):
+    prob = inputs.make_masked(5, 200, 272, 384, seed=31, masked_m=[0, 200, 1, 128, 129])
+    ref = oracle.gemm_masked(prob.a, prob.sa, prob.b, prob.sb, prob.masked_m, prob.G,
+                             prob.M_max, prob.N, prob.K)
+    d = H.run_masked(prob, expected_m=expected_m)
+    check_status()
+    got = H.bf16_bits_to_f64(d)
+    valid = ~np.isnan(ref)
+    H.assert_close(got[valid], ref[valid], "masked small")
+    assert H.untouched(d)[~valid].all(), "rows at or beyond masked_m were written"
+
+
+@pytest.mark.parametrize("mw,bn", [(1, 64), (1, 224), (2, 64), (2, 128)])
+def test_masked_forced_shapes(mw, bn):
+    prob = inputs.make_masked(3, 300, 256, 256, seed=32 + bn, masked_m=[300, 0, 129])
+    ref = oracle.gemm_masked(prob.a, prob.sa, prob.b, prob.sb, prob.masked_m, prob.G,
+                             prob.M_max, prob.N, prob.K)
+    fp8.force_config(128 * mw, bn)
+    try:
+        d = H.run_masked(prob)
+    finally:
+        fp8.force_config(0, 0)
+    check_status()
+    valid = ~np.isnan(ref)
+    H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], f"masked mw{mw} bn{bn}")
+    assert H.untouched(d)[~valid].all()
+
+
+def test_masked_all_empty_and_out_of_range():
+    prob = inputs.make_masked(3, 64, 128, 128, seed=33, masked_m=[0, 0, 0])
+    d = H.run_masked(prob)
+    check_status()
+    assert H.untouched(d).all()
+    prob.masked_m[1] = 500  # beyond M_max: clamped, flagged
+    d = H.run_masked(prob)
+    assert fp8.get_device_status() == 7
+    ref = oracle.gemm_masked(prob.a, prob.sa, prob.b, prob.sb, torch.tensor([0, 64, 0],
+                             dtype=torch.int32), 3, 64, 128, 128)
+    got = H.bf16_bits_to_f64(d)
+    H.assert_close(got[1], ref[1], "masked clamped")
+
+
+# --------------------------------------------------------------------- full size
+
+
+def _sample(rng, n, hi):
+    return rng.integers(0, hi, n)
+
+
+@pytest.mark.parametrize("name", ["dense_128x128x512", "dense_decode_64x2112x7168",
+                                  "dense_prefill_4096x7168x2048", "dense_prefill_256x7168x2048"])
+def test_full_size_dense(name):
+    prob = inputs.make_workload(name)
+    d = H.run_dense(prob)
+    check_status()
+    got = H.bf16_bits_to_f64(d)
+    rng = np.random.default_rng(1)
+    rows = np.concatenate([_sample(rng, 3000, prob.M), np.full(prob.N, prob.M - 1)])
+    cols = np.concatenate([_sample(rng, 3000, prob.N), np.arange(prob.N)])
+    ref = oracle.gemm_dense_sampled(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K,
+                                    rows, cols)
+    H.assert_close(got[rows, cols], ref, name)
+    d2 = H.run_dense(prob)
+    assert torch.equal(d.view(torch.int16), d2.view(torch.int16))
+
+
+def test_full_size_contiguous():
+    prob = inputs.make_workload("contiguous_8x4096x7168")
+    d = H.run_contiguous(prob)
+    check_status()
+    got = H.bf16_bits_to_f64(d)
+    mi = prob.m_indices.numpy()
+    valid_rows = np.nonzero(mi >= 0)[0]
+    rng = np.random.default_rng(2)
+    rows = valid_rows[rng.integers(0, len(valid_rows), 4000)]
+    cols = _sample(rng, 4000, prob.N)
+    # whole first and last row of every expert
+    starts = np.nonzero(np.diff(np.concatenate([[-2], mi])) != 0)[0]
+    edge_rows = []
+    for s in starts:
+        if mi[s] >= 0:
+            e = mi[s]
+            last = s + int(np.sum(mi[s:s + 9000] == e)) - 1
+            edge_rows += [s, last]
+    rows = np.concatenate([rows, np.repeat(edge_rows, prob.N)])
+    cols = np.concatenate([cols, np.tile(np.arange(prob.N), len(edge_rows))])
+    ref = oracle.gemm_contiguous_sampled(prob.a, prob.sa, prob.b, prob.sb, prob.m_indices,
+                                         prob.num_groups, prob.M_sum, prob.N, prob.K, rows, cols)
+    H.assert_close(got[rows, cols], ref, "contiguous full")
+    assert H.untouched(d)[mi < 0].all(), "padding rows were written"
+
+
+@pytest.mark.parametrize("name", ["masked_16x256_4096x7168", "masked_16x256_7168x2048"])
+def test_full_size_masked(name):
+    prob = inputs.make_workload(name)
+    expected_m = max(1, int(prob.masked_m.float().mean().item()))
+    d = H.run_masked(prob, expected_m=expected_m)
+    check_status()
+    got = H.bf16_bits_to_f64(d)
+    mm = prob.masked_m.numpy()
+    rng = np.random.default_rng(3)
+    act = np.nonzero(mm > 0)[0]
+    groups = act[rng.integers(0, len(act), 4000)]
+    rows = rng.integers(0, 1 << 30, 4000) % mm[groups]
+    cols = _sample(rng, 4000, prob.N)
+    last_g = act
+    groups = np.concatenate([groups, np.repeat(last_g, prob.N)])
+    rows = np.concatenate([rows, np.repeat(mm[last_g] - 1, prob.N)])
+    cols = np.concatenate([cols, np.tile(np.arange(prob.N), len(last_g))])
+    ref = oracle.gemm_masked_sampled(prob.a, prob.sa, prob.b, prob.sb, prob.masked_m, prob.G,
+                                     prob.M_max, prob.N, prob.K, groups, rows, cols)
+    H.assert_close(got[groups, rows, cols], ref, name)
+    unt = H.untouched(d)
+    for g in range(prob.G):
+        assert unt[g, mm[g]:].all(), f"group {g}: rows beyond masked_m written"

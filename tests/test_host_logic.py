@@ -1,0 +1,153 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports
+every symbol include/fp8_nt.h declares, validates arguments before touching the
+device, and chooses tile configurations deterministically."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_fine_grained_nt_b200 as fp8
+from fp8_fine_grained_nt_b200 import binding, inputs
+from tests.conftest import ROOT, read_golden
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_fine_grained_nt_b200 import build
+    build.build()
+    return binding.load_library()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "fp8_nt.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:int|const char \*|void)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function(lib):
+    names = header_functions()
+    assert "gemm_fp8_fp8_bf16_nt" in names and len(names) >= 11
+    handle = ctypes.CDLL(binding.library_path())
+    for name in names:
+        assert hasattr(handle, name), f"{name} declared in fp8_nt.h but not exported"
+
+
+def test_tma_aligned_size(lib):
+    assert fp8.get_tma_aligned_size(0, 4) == 0
+    assert fp8.get_tma_aligned_size(1, 4) == 4
+    assert fp8.get_tma_aligned_size(64, 4) == 64
+    assert fp8.get_tma_aligned_size(65, 4) == 68
+    assert fp8.get_tma_aligned_size(3, 2) == 8
+    assert fp8.get_tma_aligned_size(17, 1) == 32
+    for x in range(0, 300, 7):
+        assert fp8.get_tma_aligned_size(x, 4) == inputs.tma_aligned_size(x, 4)
+    assert lib.get_tma_aligned_size(5, 3) < 0
+    assert lib.get_tma_aligned_size(-1, 4) < 0
+
+
+def test_contiguous_alignment(lib):
+    assert fp8.get_m_alignment_for_contiguous_layout() == inputs.M_ALIGNMENT_CONTIGUOUS == 128
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert fp8.status_string(code) not in ("", "unknown status")
+    assert fp8.status_string(99) == "unknown status"
+
+
+def test_host_checks_return_before_any_device_work(lib):
+    # fake, never dereferenced pointers: the host rejects these before launch
+    p = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10008)
+    g = lib.gemm_fp8_fp8_bf16_nt
+    assert g(p, p, p, p, p, 128, 128, 100, None) == 3   # K % 128
+    assert g(p, p, p, p, p, 128, 100, 128, None) == 3   # N % 8
+    assert g(p, p, p, p, p, 128, 128, 0, None) == 3     # K == 0
+    assert g(p, p, p, p, p, -1, 128, 128, None) == 1
+    assert g(p, p, p, p, p, 0, 128, 128, None) == 0     # empty: nothing to do
+    assert g(None, p, p, p, p, 128, 128, 128, None) == 1
+    assert g(p, p, mis, p, p, 128, 128, 128, None) == 2
+    c = lib.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous
+    assert c(p, p, p, p, p, p, 0, 128, 128, 128, None) == 1     # no groups
+    assert c(p, p, p, p, p, p, 2, 100, 128, 128, None) == 3     # M_sum not aligned
+    assert c(p, p, p, p, p, None, 2, 128, 128, 128, None) == 1  # no m_indices
+    m = lib.m_grouped_gemm_fp8_fp8_bf16_nt_masked
+    assert m(p, p, p, p, p, p, 0, 128, 128, 128, 0, None) == 1
+    assert m(p, p, p, p, p, p, 2, 128, 128, 128, -1, None) == 1
+    assert m(p, p, p, p, p, p, 5000, 128, 128, 128, 0, None) == 3
+    assert m(p, p, p, p, p, mis, 2, 128, 128, 128, 0, None) == 2
+
+
+def test_block_n_example_tile_counts(lib):
+    """The SM-fill example of the DeepGEMM README: BLOCK_N 128 -> 112 tiles,
+    BLOCK_N 112 -> 128 tiles for M=256, N=7168."""
+    rows = read_golden("block_n_example.txt")
+    try:
+        for M, N, bm, bn, tiles, sms in (map(int, r) for r in rows):
+            fp8.force_config(bm, bn)
+            cfg = fp8.select_config(fp8.KIND_DENSE, M, N, 2048, num_sms=sms)
+            assert (cfg["block_m"], cfg["block_n"], cfg["num_tiles"]) == (bm, bn, tiles)
+    finally:
+        fp8.force_config(0, 0)
+    # unforced on the same 132-SM part, the selector fills more SMs than 112
+    cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=132)
+    assert cfg["num_tiles"] <= 132 and cfg["num_tiles"] >= 128
+
+
+def test_selector_fills_b200_for_prefill_shapes(lib):
+    cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=148)
+    assert cfg["num_tiles"] <= 148 and cfg["num_tiles"] >= 128
+    assert cfg["block_n"] % 16 == 0 and cfg["block_n"] & (cfg["block_n"] - 1) != 0
+    cfg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
+    waves = -(-cfg["num_tiles"] // 148)
+    assert cfg["num_tiles"] / (waves * 148) > 0.95
+
+
+def test_selector_invariants_and_determinism(lib):
+    shapes = [(fp8.KIND_DENSE, m, n, k, 1, 0)
+              for m in (1, 64, 128, 300, 4096) for n in (8, 16, 2112, 7168) for k in (128, 7168)]
+    shapes += [(fp8.KIND_CONTIGUOUS, 128 * 40, 4096, 7168, 8, 0),
+               (fp8.KIND_MASKED, 256, 4096, 7168, 16, 0),
+               (fp8.KIND_MASKED, 256, 7168, 2048, 16, 100),
+               (fp8.KIND_MASKED, 256, 7168, 2048, 1024, 0)]
+    for kind, M, N, K, G, em in shapes:
+        a = fp8.select_config(kind, M, N, K, G, em, 148)
+        b = fp8.select_config(kind, M, N, K, G, em, 148)
+        assert a == b
+        assert a["block_m"] in (128, 256) and a["block_n"] % 16 == 0
+        assert 16 <= a["block_n"] <= 256 and (a["block_m"] == 128 or a["block_n"] <= 128)
+        assert a["stages"] >= 2 and a["sf_stages"] >= a["stages"]
+        assert a["smem_bytes"] <= 232448
+        assert a["tmem_cols"] >= 2 * (a["block_m"] // 128) * a["block_n"]
+        assert a["tmem_cols"] <= 512 and a["tmem_cols"] & (a["tmem_cols"] - 1) == 0
+        assert 1 <= a["grid"] <= 148
+        if kind == fp8.KIND_CONTIGUOUS:
+            assert a["block_m"] == 128
+
+
+def test_force_config_rejects_unbuilt_shapes(lib):
+    with pytest.raises(fp8.Fp8NtError):
+        fp8.force_config(128, 120)
+    with pytest.raises(fp8.Fp8NtError):
+        fp8.force_config(256, 256)
+    fp8.force_config(0, 0)
+
+
+def test_num_sms_bound(lib):
+    try:
+        fp8.set_num_sms(100)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=0)
+        assert cfg["grid"] <= 100
+    finally:
+        fp8.set_num_sms(0)
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    t = torch.zeros(128, 128, dtype=torch.uint8)
+    s = torch.zeros(1, 128, dtype=torch.float32)
+    with pytest.raises((ValueError, TypeError)):
+        fp8.gemm_fp8_fp8_bf16_nt(t, s, t, s, torch.zeros(128, 128, dtype=torch.bfloat16))
