@@ -226,29 +226,33 @@ def profiled_traffic(kernel_tag: str):
 
 
 def oracle_sample(cases: list[Case], budget_s: float, seed: int = 0) -> dict:
-    """Time the oracle on sampled output elements of every workload, in
-    proportion to its FLOP, for about budget_s seconds."""
+    """Time the oracle on sampled output elements of every workload, each
+    workload's share of elements proportional to its share of the step's FLOP,
+    in rounds until about budget_s seconds have been spent."""
     import oracle
     rng = np.random.default_rng(seed)
     total_flops = sum(c.flops for c in cases)
-    per_elem = {c.name: 2.0 * c.prob.K for c in cases}
-    # calibrate on a small batch of the largest case
-    big = max(cases, key=lambda c: c.flops)
-    t0 = time.time()
-    done_flops = _oracle_elems(big, 256, rng) * per_elem[big.name]
-    calib = max(time.time() - t0, 1e-3)
-    rate = done_flops / calib
-    start = time.time()
     flops = 0.0
     elems = 0
-    for c in cases:
-        share = c.flops / total_flops
-        n = int(max(32, share * budget_s * rate / per_elem[c.name]))
-        k = _oracle_elems(c, n, rng)
-        flops += k * per_elem[c.name]
-        elems += k
-    dt = time.time() - start
-    return {"flops": flops, "seconds": dt, "elements": elems, "cores": oracle.num_threads()}
+    batch = 64  # elements of the largest-FLOP workload per round, grown adaptively
+    start = time.time()
+    while True:
+        t0 = time.time()
+        for c in cases:
+            n = max(1, int(round(batch * c.flops / total_flops * len(cases))))
+            k = _oracle_elems(c, n, rng)
+            flops += k * 2.0 * c.prob.K
+            elems += k
+        dt = time.time() - t0
+        spent = time.time() - start
+        if spent >= budget_s:
+            break
+        if dt < 0.5:
+            batch *= 2
+        elif spent + dt > budget_s * 1.2:
+            batch = max(1, int(batch * (budget_s - spent) / dt))
+    return {"flops": flops, "seconds": time.time() - start, "elements": elems,
+            "cores": oracle.num_threads()}
 
 
 def _oracle_elems(c: Case, n: int, rng) -> int:
@@ -281,6 +285,15 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device: str = "cuda") -> float:
+    """The maximum of `value` over all ranks (value itself when world == 1)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 def init_dist(world: int, backend: str):
@@ -358,7 +371,6 @@ def run_gpu(args):
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    time.sleep(0.3)
     start.record(stream)
     for s in range(args.steps):
         for i, c in enumerate(cases):
@@ -372,10 +384,7 @@ def run_gpu(args):
     elapsed_ms = start.elapsed_time(end)
     per_case_ms = [sum(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)) / args.steps
                    for i in range(len(cases))]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_per_step = elapsed_ms / args.steps
     step_flops = sum(c.flops for c in cases)
     value = world * step_flops / (ms_per_step * 1e-3) / 1e12
@@ -397,10 +406,7 @@ def run_gpu(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
     h2d = sum(c.h2d_bytes() for c in cases)
     d2h = sum(c.d2h_bytes() for c in cases)
@@ -483,8 +489,8 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)

@@ -9,7 +9,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include "../../include/fp8_nt.h"
+#include "fp8_nt.h"
 #include "launch.h"
 #include "params.h"
 

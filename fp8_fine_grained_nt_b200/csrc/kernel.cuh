@@ -194,51 +194,90 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, volat
         wait_slow(a, parity, abort_flag, p.status, p.timeout_ns, false);
 }
 
-__device__ __forceinline__ float pick_scale(int c, int t1, int t2, float s0, float s1, float s2)
+// Columns [c0, c0 + W) of one TMEM group into registers (W = 32, 16 or 8).
+template <int W>
+__device__ __forceinline__ void tmem_ld_group(uint32_t taddr, float (&v)[32])
 {
-    return c < t1 ? s0 : (c < t2 ? s1 : s2);
+    if constexpr (W == 32)
+        tmem_ld32(taddr, v);
+    else if constexpr (W == 16)
+        tmem_ld16(taddr, v);
+    else
+        tmem_ld8(taddr, v);
 }
 
+// A thread's NC columns are read from TMEM in groups: NC / 32 groups of 32,
+// then a 16-column and / or an 8-column tail.
 template <int NC>
-__device__ __forceinline__ void fma_chunk8(float (&acc)[NC], int c0, const float *v, float s)
-{
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        acc[c0 + j] = fmaf(v[j], s, acc[c0 + j]);
-}
-
-// acc[c] += P[row, col0 + c] * scale(c) for c in [0, NC): the promotion of
-// one K block's partial.  TMEM is read 16 columns at a time, the next group
-// in flight while the current one is multiplied in.
-template <int NC>
-__device__ __forceinline__ void promote(float (&acc)[NC], uint32_t taddr, float s0, float s1,
-                                        float s2, int t1, int t2)
-{
-    constexpr int NG = NC / 16;
-    constexpr bool TAIL8 = (NC % 16) != 0;
-    float buf[2][16];
-    if constexpr (NG == 0) {
-        tmem_ld8(taddr, buf[0]);
-        tmem_wait_ld(buf[0]);
-        fma_chunk8<NC>(acc, 0, buf[0], pick_scale(0, t1, t2, s0, s1, s2));
-    } else {
-        tmem_ld16(taddr, buf[0]);
-        tmem_wait_ld(buf[0]);
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            const bool more = (g + 1 < NG) || TAIL8;
-            if (g + 1 < NG)
-                tmem_ld16(taddr + (g + 1) * 16, buf[(g + 1) & 1]);
-            else if (TAIL8)
-                tmem_ld8(taddr + NG * 16, buf[(g + 1) & 1]);
-            fma_chunk8<NC>(acc, g * 16, buf[g & 1], pick_scale(g * 16, t1, t2, s0, s1, s2));
-            fma_chunk8<NC>(acc, g * 16 + 8, buf[g & 1] + 8, pick_scale(g * 16 + 8, t1, t2, s0, s1, s2));
-            if (more)
-                tmem_wait_ld(buf[(g + 1) & 1]);
-        }
-        if constexpr (TAIL8)
-            fma_chunk8<NC>(acc, NG * 16, buf[NG & 1], pick_scale(NG * 16, t1, t2, s0, s1, s2));
+struct Groups {
+    static constexpr int n32 = NC / 32;
+    static constexpr bool t16 = (NC % 32) >= 16;
+    static constexpr bool t8 = (NC % 16) == 8;
+    static constexpr int count = n32 + (t16 ? 1 : 0) + (t8 ? 1 : 0);
+    __host__ __device__ static constexpr int width(int g) { return g < n32 ? 32 : (t16 && g == n32 ? 16 : 8); }
+    __host__ __device__ static constexpr int offset(int g)
+    {
+        return g <= n32 ? 32 * g : 32 * n32 + (t16 ? 16 : 0);
     }
+};
+
+// acc[c0 + j] += v[j] * s for j in [0, W), two columns per instruction.
+template <int NC, int W>
+__device__ __forceinline__ void fma_group_uniform(float (&acc)[NC], int c0, const float (&v)[32],
+                                                  uint64_t s2)
+{
+#pragma unroll
+    for (int j = 0; j < W; j += 2)
+        ffma2(acc[c0 + j], acc[c0 + j + 1], v[j], v[j + 1], s2);
+}
+
+// As above with the scale chosen per 8 columns: local columns before t use
+// s_lo, the rest s_hi.  A thread owns at most 128 columns, so they span at
+// most two 128-wide scale blocks.
+template <int NC, int W>
+__device__ __forceinline__ void fma_group_split(float (&acc)[NC], int c0, const float (&v)[32],
+                                                float s_lo, float s_hi, int t)
+{
+#pragma unroll
+    for (int j = 0; j < W; j += 8) {
+        const uint64_t s2 = splat2(c0 + j < t ? s_lo : s_hi);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+            ffma2(acc[c0 + j + i], acc[c0 + j + i + 1], v[j + i], v[j + i + 1], s2);
+    }
+}
+
+template <int NC, bool SPLIT, int G>
+__device__ __forceinline__ void promote_from(float (&acc)[NC], uint32_t taddr, float (&buf)[2][32],
+                                             float s_lo, float s_hi, uint64_t s2, int t)
+{
+    using Gs = Groups<NC>;
+    if constexpr (G < Gs::count) {
+        if constexpr (G + 1 < Gs::count)
+            tmem_ld_group<Gs::width(G + 1)>(taddr + Gs::offset(G + 1), buf[(G + 1) & 1]);
+        if constexpr (SPLIT)
+            fma_group_split<NC, Gs::width(G)>(acc, Gs::offset(G), buf[G & 1], s_lo, s_hi, t);
+        else
+            fma_group_uniform<NC, Gs::width(G)>(acc, Gs::offset(G), buf[G & 1], s2);
+        if constexpr (G + 1 < Gs::count)
+            tmem_wait_ld(buf[(G + 1) & 1]);
+        promote_from<NC, SPLIT, G + 1>(acc, taddr, buf, s_lo, s_hi, s2, t);
+    }
+}
+
+// acc[c] += P[row, col0 + c] * scale(c), c in [0, NC): one K block's
+// promotion.  The next TMEM group's load is in flight while the current
+// group is multiplied in.  SPLIT: the columns straddle a scale-block boundary
+// at local column t.
+template <int NC, bool SPLIT>
+__device__ __forceinline__ void promote(float (&acc)[NC], uint32_t taddr, float s_lo, float s_hi,
+                                        int t)
+{
+    float buf[2][32];
+    const uint64_t s2 = splat2(s_lo);
+    tmem_ld_group<Groups<NC>::width(0)>(taddr, buf[0]);
+    tmem_wait_ld(buf[0]);
+    promote_from<NC, SPLIT, 0>(acc, taddr, buf, s_lo, s_hi, s2, t);
 }
 
 template <int MW, int BN>
@@ -471,8 +510,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float *sbt = sb_tile + slot * MAX_SB_BLOCKS * pitch;
             const bool active = (MW == 1) || (half * HALF_M < ti.rows);
             const int cbase = ti.n0 + col0;
-            const int t1 = ((ti.n0 >> 7) + 1) * 128 - cbase;
-            const int t2 = t1 + 128;
+            // scale blocks of this thread's columns: lo = block of its first
+            // column (relative to the tile's first block), t = local column
+            // where the next block starts
+            const int lo = (cbase >> 7) - (ti.n0 >> 7);
+            const int t_split = ((cbase >> 7) + 1) * 128 - cbase;
+            const bool split = t_split < NC;
             float acc[NC];
 #pragma unroll
             for (int c = 0; c < NC; ++c)
@@ -490,12 +533,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 const float sa_v = sf_ring[f * MW * HALF_M + row_in_tile];
-                const float s0 = sa_v * sbt[kb];
-                const float s1 = sa_v * sbt[pitch + kb];
-                const float s2 = sa_v * sbt[2 * pitch + kb];
-                if (active)
-                    promote<NC>(acc, tmem_base + lane_off + (uint32_t)(buf * T::BUF_COLS + half * BN + col0),
-                                s0, s1, s2, t1, t2);
+                const float s_lo = sa_v * sbt[lo * pitch + kb];
+                const uint32_t taddr =
+                    tmem_base + lane_off + (uint32_t)(buf * T::BUF_COLS + half * BN + col0);
+                if (active) {
+                    if (split)
+                        promote<NC, true>(acc, taddr, s_lo, sa_v * sbt[(lo + 1) * pitch + kb],
+                                          t_split);
+                    else
+                        promote<NC, false>(acc, taddr, s_lo, s_lo, NC);
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
