@@ -53,7 +53,7 @@ class Fp8NtError(RuntimeError):
 
 class DgConfig(ctypes.Structure):
     _fields_ = [("block_m", ctypes.c_int), ("block_n", ctypes.c_int),
-                ("stages", ctypes.c_int), ("sf_stages", ctypes.c_int),
+                ("stages", ctypes.c_int),
                 ("num_tiles", ctypes.c_int), ("grid", ctypes.c_int),
                 ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int)]
 

@@ -187,17 +187,14 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int sms, int *tiles_ou
     return waves * tile;
 }
 
-int plan_for(const Problem &pb, int mw, int bn, int max_smem, int *stages, int *sf_stages,
-             SmemPlan *plan)
+int plan_for(const Problem &pb, int mw, int bn, int max_smem, int *stages, SmemPlan *plan)
 {
     const int nkb = pb.K / 128;
     const int prefix_ints = pb.kind == DG_KIND_MASKED ? 2 * pb.groups + 1 : 0;
     for (int s = kMaxStages; s >= kMinStages; --s) {
-        const int sf = s + 4;
-        SmemPlan p = make_smem_plan(mw, bn, s, sf, nkb, prefix_ints);
+        SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints);
         if ((int)p.total + 1024 <= max_smem) {
             *stages = s;
-            *sf_stages = sf;
             *plan = p;
             return DG_OK;
         }
@@ -216,9 +213,9 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
             continue;
         if (pb.kind == DG_KIND_CONTIGUOUS && c.mw != 1)
             continue; // a 256-row tile could straddle two 128-aligned experts
-        int st, sf;
+        int st;
         SmemPlan p;
-        if (plan_for(pb, c.mw, c.bn, max_smem, &st, &sf, &p) != DG_OK)
+        if (plan_for(pb, c.mw, c.bn, max_smem, &st, &p) != DG_OK)
             continue;
         const double cost = estimate_cycles(pb, c.mw, c.bn, sms, nullptr);
         // ties: wider tile first (fewer re-reads of A), then one M half
@@ -232,8 +229,8 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     }
     if (!best)
         return DG_ERR_UNSUPPORTED_SHAPE;
-    int st, sf;
-    plan_for(pb, best->mw, best->bn, max_smem, &st, &sf, plan);
+    int st;
+    plan_for(pb, best->mw, best->bn, max_smem, &st, plan);
     const int bm = best->mw * 128;
     long tiles;
     if (pb.kind == DG_KIND_MASKED)
@@ -245,7 +242,6 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     cfg->block_m = bm;
     cfg->block_n = best->bn;
     cfg->stages = st;
-    cfg->sf_stages = sf;
     cfg->num_tiles = (int)tiles;
     cfg->grid = (int)(tiles < sms ? tiles : sms);
     if (cfg->grid < 1)
@@ -304,18 +300,14 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     const int groups = pb.kind == DG_KIND_DENSE ? 1 : pb.groups;
     const int ld_sa = get_tma_aligned_size(pb.M, 4);
 
-    CUtensorMap tmap_a, tmap_b, tmap_sa;
+    CUtensorMap tmap_a, tmap_b;
     const long a_rows = pb.kind == DG_KIND_MASKED ? (long)groups * pb.M : pb.M;
     const long b_rows = (long)groups * pb.N;
-    const long sa_rows = pb.kind == DG_KIND_MASKED ? (long)groups * nkb : nkb;
     if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, a_rows, pb.K, 128,
                            128, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
         return st;
     if ((st = make_tmap_2d(&tmap_b, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, b_rows, pb.K, 128,
                            cfg.block_n, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-        return st;
-    if ((st = make_tmap_2d(&tmap_sa, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ld_sa, sa_rows, ld_sa,
-                           128, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
         return st;
 
     Params p;
@@ -331,8 +323,9 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     p.n_blocks = ceil_div(pb.N, cfg.block_n);
     p.num_tiles = cfg.num_tiles;
     p.stages = cfg.stages;
-    p.sf_stages = cfg.sf_stages;
     p.plan = plan;
+    p.sa = sa;
+    p.ld_sa = ld_sa;
     p.sb = sb;
     p.m_indices = m_indices;
     p.masked_m = masked_m;
@@ -343,7 +336,6 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     LaunchArgs args;
     args.tmap_a = &tmap_a;
     args.tmap_b = &tmap_b;
-    args.tmap_sa = &tmap_sa;
     args.params = &p;
     args.grid = cfg.grid;
     args.smem_bytes = cfg.smem_bytes;

@@ -25,7 +25,7 @@ cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN)(const LaunchArgs &args)
     if (err != cudaSuccess)
         return err;
     kernel<<<args.grid, NUM_THREADS, args.smem_bytes, args.stream>>>(*args.tmap_a, *args.tmap_b,
-                                                                     *args.tmap_sa, *args.params);
+                                                                     *args.params);
     return cudaGetLastError();
 }
 

@@ -10,14 +10,17 @@
 //
 // Roles (384 threads, one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: A / B tiles into a multi-stage shared-memory
-//               ring, the tile's LHS scales into a scale ring (TMA), the
-//               tile's RHS scales into a per-tile slot (cp.async).  The
-//               README's data-movement warpgroup, reduced to one warp.
+//               ring (the A and B copies of a stage issued by two lanes in one
+//               instruction), the tile's RHS scales into a per-tile slot
+//               (cp.async).  The README's data-movement warpgroup, reduced to
+//               one warp.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer: one
-//               128-K block per MMA group into one of two TMEM buffers, fresh
+//               128-K block per MMA group into a ring of TMEM buffers, fresh
 //               accumulation per block so each block's partial stays separable.
-//   warps 4-11  promotion epilogue: tcgen05.ld of a block's partial, FMA with
-//               sa*sb into FP32 registers, BF16 conversion and store at tile end.
+//   warps 4-11  promotion epilogue: tcgen05.ld of the blocks' partials, FMA
+//               with sa*sb into FP32 registers (sa read from global memory a
+//               few blocks ahead), BF16 conversion and a coalesced store at
+//               tile end.
 // Warps 2-3 only help with set-up (masked tile counts).
 //
 // Tile shape: BLOCK_M = 128 * MW rows (MW = 2 issues two M=128 MMAs that share
@@ -39,13 +42,23 @@ struct KernelTraits {
     static_assert(MW == 1 || BN <= 128, "two M halves need BN <= 128 (TMEM and registers)");
     static constexpr int BLOCK_M = MW * HALF_M;
     static constexpr int BUF_COLS = MW * BN;                 // TMEM columns per K-block buffer
-    static constexpr int TMEM_NEED = 2 * BUF_COLS;
+    // ring of K-block partial buffers in TMEM: as many as fit, at most 16
+    static constexpr int NBUF = (512 / BUF_COLS) < MAX_TMEM_BUFS ? (512 / BUF_COLS) : MAX_TMEM_BUFS;
+    static constexpr int TMEM_NEED = NBUF * BUF_COLS;
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                    : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
     static constexpr int COLS_PER_THREAD = (MW == 1) ? BN / 2 : BN;
+    // a thread's whole partial fits one 64-register batch: the next K block's
+    // partial can then be in flight while the current one is multiplied in
+    static constexpr bool PREFETCH = COLS_PER_THREAD <= 64;
+    // K blocks promoted per epilogue step: their partials (GROUP x
+    // COLS_PER_THREAD <= 64 registers) are loaded with one wait and their
+    // buffers released together, which amortises the per-block handshake.
+    static constexpr int GROUP_BY_REGS = PREFETCH ? 64 / COLS_PER_THREAD : 1;
+    static constexpr int GROUP = GROUP_BY_REGS < NBUF / 2 ? GROUP_BY_REGS : (NBUF / 2 > 0 ? NBUF / 2 : 1);
     static constexpr uint32_t A_HALF_BYTES = HALF_M * BLOCK_K;
     static constexpr uint32_t B_BYTES = BN * BLOCK_K;
-    static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
+    static_assert(NBUF >= 2 && NBUF <= MAX_TMEM_BUFS && TMEM_NEED <= 512, "TMEM holds 512 columns");
     static_assert(COLS_PER_THREAD % 8 == 0, "epilogue works in 8-column chunks");
 };
 
@@ -79,7 +92,7 @@ struct TileInfo {
     int rows;    // rows of the tile that hold valid data (<= BLOCK_M)
     int a_row0;  // row coordinate of the tile in A's 2-D tensor map
     int b_row0;  // row coordinate in B's 2-D tensor map
-    int sa_y0;   // row of sa's 2-D tensor map holding K block 0 of this group
+    int sa_y0;   // row of sa ([G*K/128][ld]) holding K block 0 of this group
     int sb_row0; // first sb row (128-column block) of the tile, group base included
     int sb_rows; // sb rows present from sb_row0 within the group (<= 3)
     int d_row0;  // row of D (all groups flattened) holding row m0
@@ -194,97 +207,85 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, volat
         wait_slow(a, parity, abort_flag, p.status, p.timeout_ns, false);
 }
 
-// Columns [c0, c0 + W) of one TMEM group into registers (W = 32, 16 or 8).
-template <int W>
-__device__ __forceinline__ void tmem_ld_group(uint32_t taddr, float (&v)[32])
+// Issue tcgen05.ld for columns [C, N) of a thread's lane into v[C..N):
+// 32-column loads, then a 16- and / or 8-column tail.  No wait.
+template <int N, int C = 0>
+__device__ __forceinline__ void tmem_issue_p(uint32_t taddr, float *v)
 {
-    if constexpr (W == 32)
-        tmem_ld32(taddr, v);
-    else if constexpr (W == 16)
-        tmem_ld16(taddr, v);
-    else
-        tmem_ld8(taddr, v);
-}
-
-// A thread's NC columns are read from TMEM in groups: NC / 32 groups of 32,
-// then a 16-column and / or an 8-column tail.
-template <int NC>
-struct Groups {
-    static constexpr int n32 = NC / 32;
-    static constexpr bool t16 = (NC % 32) >= 16;
-    static constexpr bool t8 = (NC % 16) == 8;
-    static constexpr int count = n32 + (t16 ? 1 : 0) + (t8 ? 1 : 0);
-    __host__ __device__ static constexpr int width(int g) { return g < n32 ? 32 : (t16 && g == n32 ? 16 : 8); }
-    __host__ __device__ static constexpr int offset(int g)
-    {
-        return g <= n32 ? 32 * g : 32 * n32 + (t16 ? 16 : 0);
+    if constexpr (C < N) {
+        constexpr int W = (N - C >= 32) ? 32 : ((N - C >= 16) ? 16 : 8);
+        if constexpr (W == 32)
+            tmem_ld32(taddr + C, *reinterpret_cast<float(*)[32]>(v + C));
+        else if constexpr (W == 16)
+            tmem_ld16(taddr + C, *reinterpret_cast<float(*)[16]>(v + C));
+        else
+            tmem_ld8p(taddr + C, v + C);
+        tmem_issue_p<N, C + W>(taddr, v);
     }
-};
-
-// acc[c0 + j] += v[j] * s for j in [0, W), two columns per instruction.
-template <int NC, int W>
-__device__ __forceinline__ void fma_group_uniform(float (&acc)[NC], int c0, const float (&v)[32],
-                                                  uint64_t s2)
-{
-#pragma unroll
-    for (int j = 0; j < W; j += 2)
-        ffma2(acc[c0 + j], acc[c0 + j + 1], v[j], v[j + 1], s2);
 }
 
-// As above with the scale chosen per 8 columns: local columns before t use
-// s_lo, the rest s_hi.  A thread owns at most 128 columns, so they span at
-// most two 128-wide scale blocks.
-template <int NC, int W>
-__device__ __forceinline__ void fma_group_split(float (&acc)[NC], int c0, const float (&v)[32],
-                                                float s_lo, float s_hi, int t)
+template <int N>
+__device__ __forceinline__ void tmem_issue(uint32_t taddr, float (&v)[64])
 {
+    tmem_issue_p<N>(taddr, v);
+}
+
+// Wait for every outstanding tcgen05.ld of this thread; all 64 registers are
+// tied to the wait so that none of them is read before it.
+__device__ __forceinline__ void tmem_wait64(float (&v)[64])
+{
+    tmem_wait_ld(*reinterpret_cast<float(*)[32]>(&v[0]));
+    reg_tie32(*reinterpret_cast<float(*)[32]>(&v[32]));
+}
+
+// acc[C0 + j] += v[j] * scale for j in [0, N), two columns per instruction.
+// SPLIT: local columns before t use s_lo, the rest s_hi (chosen per 8
+// columns; a thread owns at most 128 columns, so they span at most two
+// 128-wide scale blocks).
+template <int NC, int C0, int N, bool SPLIT>
+__device__ __forceinline__ void fma_range(float (&acc)[NC], const float (&v)[64], float s_lo,
+                                          float s_hi, int t)
+{
+    const uint64_t s2_lo = splat2(s_lo);
 #pragma unroll
-    for (int j = 0; j < W; j += 8) {
-        const uint64_t s2 = splat2(c0 + j < t ? s_lo : s_hi);
+    for (int j = 0; j < N; j += 8) {
+        const uint64_t s2 = SPLIT ? splat2(C0 + j < t ? s_lo : s_hi) : s2_lo;
 #pragma unroll
         for (int i = 0; i < 8; i += 2)
-            ffma2(acc[c0 + j + i], acc[c0 + j + i + 1], v[j + i], v[j + i + 1], s2);
+            ffma2(acc[C0 + j + i], acc[C0 + j + i + 1], v[j + i], v[j + i + 1], s2);
     }
 }
 
-template <int NC, bool SPLIT, int G>
-__device__ __forceinline__ void promote_from(float (&acc)[NC], uint32_t taddr, float (&buf)[2][32],
-                                             float s_lo, float s_hi, uint64_t s2, int t)
-{
-    using Gs = Groups<NC>;
-    if constexpr (G < Gs::count) {
-        if constexpr (G + 1 < Gs::count)
-            tmem_ld_group<Gs::width(G + 1)>(taddr + Gs::offset(G + 1), buf[(G + 1) & 1]);
-        if constexpr (SPLIT)
-            fma_group_split<NC, Gs::width(G)>(acc, Gs::offset(G), buf[G & 1], s_lo, s_hi, t);
-        else
-            fma_group_uniform<NC, Gs::width(G)>(acc, Gs::offset(G), buf[G & 1], s2);
-        if constexpr (G + 1 < Gs::count)
-            tmem_wait_ld(buf[(G + 1) & 1]);
-        promote_from<NC, SPLIT, G + 1>(acc, taddr, buf, s_lo, s_hi, s2, t);
-    }
-}
-
-// acc[c] += P[row, col0 + c] * scale(c), c in [0, NC): one K block's
-// promotion.  The next TMEM group's load is in flight while the current
-// group is multiplied in.  SPLIT: the columns straddle a scale-block boundary
-// at local column t.
+// acc[c] += v[c] * scale(c) for all NC columns, v a pointer into a
+// register array (compile-time offset after unrolling).
 template <int NC, bool SPLIT>
-__device__ __forceinline__ void promote(float (&acc)[NC], uint32_t taddr, float s_lo, float s_hi,
-                                        int t)
+__device__ __forceinline__ void fma_all_p(float (&acc)[NC], const float *v, float s_lo, float s_hi,
+                                          int t)
 {
-    float buf[2][32];
-    const uint64_t s2 = splat2(s_lo);
-    tmem_ld_group<Groups<NC>::width(0)>(taddr, buf[0]);
-    tmem_wait_ld(buf[0]);
-    promote_from<NC, SPLIT, 0>(acc, taddr, buf, s_lo, s_hi, s2, t);
+    const uint64_t s2_lo = splat2(s_lo);
+#pragma unroll
+    for (int j = 0; j < NC; j += 8) {
+        const uint64_t s2 = SPLIT ? splat2(j < t ? s_lo : s_hi) : s2_lo;
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+            ffma2(acc[j + i], acc[j + i + 1], v[j + i], v[j + i + 1], s2);
+    }
+}
+
+template <int NC, int C0, int N>
+__device__ __forceinline__ void fma_range_any(float (&acc)[NC], const float (&v)[64], float s_lo,
+                                              float s_hi, int t, bool split)
+{
+    if (split)
+        fma_range<NC, C0, N, true>(acc, v, s_lo, s_hi, t);
+    else
+        fma_range<NC, C0, N, false>(acc, v, s_lo, s_hi, t);
 }
 
 template <int MW, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b,
-                    const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ Params p)
+                    const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ Params p)
 {
     using T = KernelTraits<MW, BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -295,21 +296,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int lane = threadIdx.x & 31;
     const SmemPlan &plan = p.plan;
     const int stages = p.stages;
-    const int sf_stages = p.sf_stages;
 
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + plan.off_bars);
     uint64_t *empty = full + stages;
-    uint64_t *sf_full = empty + stages;
-    uint64_t *sf_empty = sf_full + sf_stages;
-    uint64_t *tmem_full = sf_empty + sf_stages;
-    uint64_t *tmem_empty = tmem_full + 2;
-    uint64_t *sb_full = tmem_empty + 2;
+    uint64_t *tmem_full = empty + stages;
+    uint64_t *tmem_empty = tmem_full + MAX_TMEM_BUFS;
+    uint64_t *sb_full = tmem_empty + MAX_TMEM_BUFS;
     uint64_t *sb_empty = sb_full + 2;
     uint64_t *mma_done = sb_empty + 2;
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + plan.off_misc);
     volatile uint32_t *abort_flag = misc + 1;
     int *prefix = reinterpret_cast<int *>(smem + plan.off_prefix);
-    float *sf_ring = reinterpret_cast<float *>(smem + plan.off_sf);
     float *sb_tile = reinterpret_cast<float *>(smem + plan.off_sb);
     const int pitch = (int)plan.sb_pitch;
 
@@ -319,13 +316,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int s = 0; s < sf_stages; ++s) {
-            mbar_init(&sf_full[s], 1);
-            mbar_init(&sf_empty[s], NUM_EPI_WARPS);
-        }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < T::NBUF; ++b) {
             mbar_init(&tmem_full[b], 1);
             mbar_init(&tmem_empty[b], NUM_EPI_WARPS);
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&sb_full[b], 32);
             mbar_init(&sb_empty[b], NUM_EPI_WARPS);
         }
@@ -336,7 +331,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
-        tma_prefetch_desc(&tmap_sa);
     }
     if (warp == 1) {
         tmem_alloc(misc, T::TMEM_COLS);
@@ -381,12 +375,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         regs_dec<REGS_PRODUCER>();
-        uint32_t stage_it = 0, sf_it = 0, tile_it = 0;
+        uint32_t stage_it = 0, tile_it = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
             const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
             if (!ti.valid)
                 continue;
+            // RHS scales of the whole tile: <= 3 rows of K/128 floats
             const int slot = tile_it & 1;
             if (!wait_bar_warp(&sb_empty[slot], ((tile_it >> 1) & 1) ^ 1, abort_flag, p))
                 break;
@@ -398,37 +393,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     cp_async_4(dst + j * pitch + kb, p.sb + (size_t)(ti.sb_row0 + j) * p.nkb + kb);
             }
             cp_async_mbar_arrive_noinc(&sb_full[slot]);
-            if (lane == 0) {
-                const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
-                const uint32_t ab_bytes = halves * T::A_HALF_BYTES + T::B_BYTES;
-                for (int kb = 0; kb < p.nkb; ++kb) {
-                    const int s = (int)(stage_it % (uint32_t)stages);
-                    if (!wait_bar(&empty[s], ((stage_it / stages) & 1) ^ 1, abort_flag, p)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *a_dst = smem + plan.off_stages + (uint32_t)s * plan.stage_bytes;
-                    uint8_t *b_dst = a_dst + plan.a_bytes;
-                    mbar_arrive_expect_tx(&full[s], ab_bytes);
-                    for (int h = 0; h < halves; ++h)
-                        tma_load_2d(a_dst + h * T::A_HALF_BYTES, &tmap_a, &full[s], kb * BLOCK_K,
-                                    ti.a_row0 + h * HALF_M);
-                    tma_load_2d(b_dst, &tmap_b, &full[s], kb * BLOCK_K, ti.b_row0);
-                    ++stage_it;
 
-                    const int f = (int)(sf_it % (uint32_t)sf_stages);
-                    if (!wait_bar(&sf_empty[f], ((sf_it / sf_stages) & 1) ^ 1, abort_flag, p)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&sf_full[f], halves * HALF_M * 4);
-                    for (int h = 0; h < halves; ++h)
-                        tma_load_2d(sf_ring + f * MW * HALF_M + h * HALF_M, &tmap_sa, &sf_full[f],
-                                    ti.m0 + h * HALF_M, ti.sa_y0 + kb);
-                    ++sf_it;
+            // A / B per K block.  Lane 0 copies B, lanes 1..halves the A
+            // halves: one instruction issues all of a stage's copies.
+            const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
+            const uint32_t ab_bytes = halves * T::A_HALF_BYTES + T::B_BYTES;
+            const bool copier = lane <= halves;
+            const CUtensorMap *my_map = lane == 0 ? &tmap_b : &tmap_a;
+            const int my_row = lane == 0 ? ti.b_row0 : ti.a_row0 + (lane - 1) * HALF_M;
+            const uint32_t my_off = lane == 0 ? plan.a_bytes : (uint32_t)(lane - 1) * T::A_HALF_BYTES;
+            for (int kb = 0; kb < p.nkb; ++kb) {
+                const int s = (int)(stage_it % (uint32_t)stages);
+                int got = 1;
+                if (lane == 0) {
+                    got = wait_bar(&empty[s], ((stage_it / stages) & 1) ^ 1, abort_flag, p) ? 1 : 0;
+                    if (got)
+                        mbar_arrive_expect_tx(&full[s], ab_bytes);
                 }
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                if (copier)
+                    tma_load_2d(smem + plan.off_stages + (uint32_t)s * plan.stage_bytes + my_off,
+                                my_map, &full[s], kb * BLOCK_K, my_row);
+                ++stage_it;
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             ++tile_it;
         }
         // Drain: every copy issued must land before the CTA exits.
@@ -437,9 +428,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t n = stage_it < (uint32_t)stages ? stage_it : (uint32_t)stages;
             for (uint32_t i = stage_it - n; i < stage_it; ++i)
                 wait_drain(&full[i % stages], (i / stages) & 1, abort_flag, p);
-            const uint32_t nf = sf_it < (uint32_t)sf_stages ? sf_it : (uint32_t)sf_stages;
-            for (uint32_t i = sf_it - nf; i < sf_it; ++i)
-                wait_drain(&sf_full[i % sf_stages], (i / sf_stages) & 1, abort_flag, p);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -459,10 +447,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    const int buf = kb_it & 1;
-                    if (!wait_bar(&tmem_empty[buf], ((kb_it >> 1) & 1) ^ 1, abort_flag, p)) {
-                        ok = false;
-                        break;
+                    // The epilogue promotes K blocks in groups of GROUP (per
+                    // tile, from K block 0) and releases a group's buffers
+                    // together, each warp in order: at the first block of a
+                    // group, waiting for the release of the group's last
+                    // buffer covers the whole group.
+                    const int gpos = kb % T::GROUP;
+                    const int buf = (int)(kb_it % T::NBUF);
+                    if (gpos == 0) {
+                        const int cnt = min(T::GROUP, p.nkb - kb);
+                        const uint32_t last = kb_it + (uint32_t)(cnt - 1);
+                        if (!wait_bar(&tmem_empty[last % T::NBUF], ((last / T::NBUF) & 1) ^ 1,
+                                      abort_flag, p)) {
+                            ok = false;
+                            break;
+                        }
                     }
                     tc_fence_after();
                     const uint32_t a_base =
@@ -476,6 +475,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                        make_sdesc(b_base + k * MMA_K), idesc, k > 0 ? 1u : 0u);
                     }
                     mma_commit(&empty[s]);
+                    // every buffer completes one phase per use (the epilogue
+                    // waits only for a group's last one)
                     mma_commit(&tmem_full[buf]);
                     ++stage_it;
                     ++kb_it;
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int half = (MW == 1) ? 0 : wg;
         const int row_in_tile = half * HALF_M + q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        uint32_t kb_it = 0, sf_it = 0, tile_it = 0;
+        uint32_t kb_it = 0, tile_it = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
             const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
@@ -511,46 +512,138 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const bool active = (MW == 1) || (half * HALF_M < ti.rows);
             const int cbase = ti.n0 + col0;
             // scale blocks of this thread's columns: lo = block of its first
-            // column (relative to the tile's first block), t = local column
-            // where the next block starts
+            // column (relative to the tile's first block), t_split = local
+            // column where the next block starts
             const int lo = (cbase >> 7) - (ti.n0 >> 7);
             const int t_split = ((cbase >> 7) + 1) * 128 - cbase;
             const bool split = t_split < NC;
+            // LHS scales of this thread's row, read from global memory four
+            // K blocks ahead of use (rows past the scale tensor's leading
+            // dimension read nothing; they are never stored)
+            const int sa_row = ti.m0 + row_in_tile;
+            const float *sa_ptr = p.sa + (size_t)ti.sa_y0 * p.ld_sa + sa_row;
+            const bool sa_ok = sa_row < p.ld_sa;
+            auto sa_load = [&](int kb) {
+                return (sa_ok && kb < p.nkb) ? __ldg(sa_ptr + (size_t)kb * p.ld_sa) : 0.0f;
+            };
+            float sa_q0 = sa_load(0), sa_q1 = sa_load(1), sa_q2 = sa_load(2), sa_q3 = sa_load(3);
+            auto scales = [&](int kb, float &s_lo, float &s_hi) {
+                const float sa_v = sa_q0;
+                sa_q0 = sa_q1;
+                sa_q1 = sa_q2;
+                sa_q2 = sa_q3;
+                sa_q3 = sa_load(kb + 4);
+                s_lo = sa_v * sbt[lo * pitch + kb];
+                s_hi = sa_v * sbt[(lo + 1) * pitch + kb];
+            };
             float acc[NC];
 #pragma unroll
             for (int c = 0; c < NC; ++c)
                 acc[c] = 0.0f;
-            for (int kb = 0; kb < p.nkb; ++kb) {
-                const int buf = kb_it & 1;
-                if (!wait_bar_warp(&tmem_full[buf], (kb_it >> 1) & 1, abort_flag, p)) {
-                    ok = false;
-                    break;
-                }
+            const uint32_t t_lane = tmem_base + lane_off + (uint32_t)(half * BN + col0);
+            auto buf_addr = [&](uint32_t it) {
+                return t_lane + (uint32_t)((int)(it % T::NBUF) * T::BUF_COLS);
+            };
+            // wait for K block `it`'s partial in TMEM
+            auto wait_full = [&](uint32_t it) {
+                const bool r = wait_bar_warp(&tmem_full[it % T::NBUF], (it / T::NBUF) & 1, abort_flag, p);
                 tc_fence_after();
-                const int f = (int)(sf_it % (uint32_t)sf_stages);
-                if (!wait_bar_warp(&sf_full[f], (sf_it / sf_stages) & 1, abort_flag, p)) {
-                    ok = false;
-                    break;
-                }
-                const float sa_v = sf_ring[f * MW * HALF_M + row_in_tile];
-                const float s_lo = sa_v * sbt[lo * pitch + kb];
-                const uint32_t taddr =
-                    tmem_base + lane_off + (uint32_t)(buf * T::BUF_COLS + half * BN + col0);
-                if (active) {
-                    if (split)
-                        promote<NC, true>(acc, taddr, s_lo, sa_v * sbt[(lo + 1) * pitch + kb],
-                                          t_split);
-                    else
-                        promote<NC, false>(acc, taddr, s_lo, s_lo, NC);
-                }
+                return r;
+            };
+            // hand K blocks [it, it + cnt) back to the MMA issuer
+            auto release = [&](uint32_t it, int cnt) {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&tmem_empty[buf]);
-                    mbar_arrive(&sf_empty[f]);
+                if (lane == 0)
+                    for (int j = 0; j < cnt; ++j)
+                        mbar_arrive(&tmem_empty[(it + j) % T::NBUF]);
+            };
+            if constexpr (T::PREFETCH) {
+                // Steps of up to GROUP K blocks: their partials are loaded
+                // together (one wait) and multiplied in while the next step's
+                // partials are in flight.
+                constexpr int G = T::GROUP;
+                float ra[64], rb[64];
+                auto load_step = [&](uint32_t it0, int cnt, float (&v)[64]) {
+                    // partials complete in issue order: the last one's
+                    // barrier covers the step
+                    if (!wait_full(it0 + cnt - 1))
+                        return false;
+                    if (active) {
+#pragma unroll
+                        for (int j = 0; j < G; ++j)
+                            if (j < cnt)
+                                tmem_issue_p<NC>(buf_addr(it0 + j), &v[j * NC]);
+                    }
+                    return true;
+                };
+                // cur holds K blocks [kb0, kb0 + cnt), loaded and waited
+                auto step = [&](float (&cur)[64], float (&nxt)[64], int kb0) {
+                    const int cnt = min(G, p.nkb - kb0);
+                    release(kb_it, cnt);
+                    const int nkb0 = kb0 + cnt;
+                    const bool more = nkb0 < p.nkb;
+                    if (more && !load_step(kb_it + cnt, min(G, p.nkb - nkb0), nxt))
+                        return false;
+#pragma unroll
+                    for (int j = 0; j < G; ++j) {
+                        if (j < cnt) {
+                            float s_lo, s_hi;
+                            scales(kb0 + j, s_lo, s_hi);
+                            if (active) {
+                                if (split)
+                                    fma_all_p<NC, true>(acc, &cur[j * NC], s_lo, s_hi, t_split);
+                                else
+                                    fma_all_p<NC, false>(acc, &cur[j * NC], s_lo, s_hi, t_split);
+                            }
+                        }
+                    }
+                    if (more && active)
+                        tmem_wait64(nxt);
+                    kb_it += cnt;
+                    return true;
+                };
+                if (!load_step(kb_it, min(G, p.nkb), ra)) {
+                    ok = false;
+                } else {
+                    if (active)
+                        tmem_wait64(ra);
+                    for (int kb0 = 0; kb0 < p.nkb; kb0 += 2 * G) {
+                        if (!step(ra, rb, kb0)) {
+                            ok = false;
+                            break;
+                        }
+                        if (kb0 + G < p.nkb && !step(rb, ra, kb0 + G)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                 }
-                ++kb_it;
-                ++sf_it;
+            } else {
+                // Two batches of at most 64 columns per K block.
+                constexpr int B0 = 64;
+                constexpr int B1 = NC - 64;
+                float r[64];
+                for (int kb = 0; kb < p.nkb; ++kb) {
+                    if (!wait_full(kb_it)) {
+                        ok = false;
+                        break;
+                    }
+                    if (active)
+                        tmem_issue<B0>(buf_addr(kb_it), r);
+                    float s_lo, s_hi;
+                    scales(kb, s_lo, s_hi);
+                    if (active) {
+                        tmem_wait64(r);
+                        fma_range_any<NC, 0, B0>(acc, r, s_lo, s_hi, t_split, split);
+                        tmem_issue<B1>(buf_addr(kb_it) + B0, r);
+                        tmem_wait64(r);
+                    }
+                    release(kb_it, 1);
+                    if (active)
+                        fma_range_any<NC, B0, B1>(acc, r, s_lo, s_hi, t_split, split);
+                    ++kb_it;
+                }
             }
             if (!ok)
                 break;
@@ -559,7 +652,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 mbar_arrive(&sb_empty[slot]);
             ++tile_it;
 
-            // ---- store this thread's row segment as BF16
+            // ---- store the tile's rows as BF16
             bool row_ok = active && row_in_tile < ti.rows;
             if (row_ok && p.kind == KIND_CONTIGUOUS) {
                 const int e = __ldg(p.m_indices + ti.d_row0 + row_in_tile);
@@ -569,16 +662,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         atomicOr(p.status, DEVERR_BAD_INDEX);
                 }
             }
-            if (row_ok) {
-                uint16_t *drow = p.D + (size_t)(ti.d_row0 + row_in_tile) * p.N + cbase;
+            // Each warp owns 32 rows; it passes them 32 columns at a time
+            // through a 2 KB shared buffer (16-byte pieces XOR-swizzled to
+            // avoid bank conflicts) so that the global writes are 64-byte
+            // row segments: 4 lanes per row, 8 rows per instruction.
+            const uint32_t row_mask = __ballot_sync(0xffffffffu, row_ok);
+            const uint32_t stg = smem_addr(smem + plan.off_out) + (uint32_t)ew * OUT_STAGE_BYTES;
+            const int warp_row0 = ti.d_row0 + half * HALF_M + q * 32;
+            const int rd_sub = lane >> 2;  // row within an 8-row group (read side)
+            const int rd_piece = lane & 3; // 16-byte piece within a 64-byte row chunk
 #pragma unroll
-                for (int c = 0; c < NC; c += 8) {
-                    if (cbase + c < p.N)
-                        st_global_v4(drow + c, pack_bf16x2(acc[c], acc[c + 1]),
-                                     pack_bf16x2(acc[c + 2], acc[c + 3]),
-                                     pack_bf16x2(acc[c + 4], acc[c + 5]),
-                                     pack_bf16x2(acc[c + 6], acc[c + 7]));
+            for (int c = 0; c < NC; c += 32) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (c + 8 * j < NC)
+                        st_shared_v4(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
+                                     pack_bf16x2(acc[c + 8 * j], acc[c + 8 * j + 1]),
+                                     pack_bf16x2(acc[c + 8 * j + 2], acc[c + 8 * j + 3]),
+                                     pack_bf16x2(acc[c + 8 * j + 4], acc[c + 8 * j + 5]),
+                                     pack_bf16x2(acc[c + 8 * j + 6], acc[c + 8 * j + 7]));
+                __syncwarp();
+                const int col = cbase + c + 8 * rd_piece;
+                const bool col_ok = (c + 8 * rd_piece < NC) && col < p.N;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = i * 8 + rd_sub;
+                    if (col_ok && ((row_mask >> r) & 1u)) {
+                        const uint4 v =
+                            ld_shared_v4(stg + r * 64 + ((rd_piece ^ ((r >> 1) & 3)) << 4));
+                        st_global_v4(p.D + (size_t)(warp_row0 + r) * p.N + col, v.x, v.y, v.z,
+                                     v.w);
+                    }
                 }
+                __syncwarp();
             }
         }
     }

@@ -12,7 +12,6 @@ namespace fp8nt {
 struct LaunchArgs {
     const CUtensorMap *tmap_a;
     const CUtensorMap *tmap_b;
-    const CUtensorMap *tmap_sa;
     const Params *params;
     int grid;
     int smem_bytes;

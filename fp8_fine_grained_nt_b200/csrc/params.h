@@ -16,6 +16,8 @@ constexpr int FIRST_EPI_WARP = 4;     // warps 4..11 run the promotion epilogue
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int MAX_SB_BLOCKS = 3;      // a BLOCK_N <= 256 tile spans at most 3 sb blocks
 constexpr int MAX_MASKED_GROUPS = 1024;
+constexpr int MAX_TMEM_BUFS = 16;      // K-block partial buffers in TMEM (ring)
+constexpr uint32_t OUT_STAGE_BYTES = 2048; // 32 rows x 32 BF16 columns per epilogue warp
 constexpr int REGS_PRODUCER = 56;     // per-thread registers after setmaxnreg
 constexpr int REGS_EPILOGUE = 224;
 constexpr int REGS_AT_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
@@ -31,10 +33,9 @@ struct SmemPlan {
     uint32_t stage_bytes;   // A (MW x 16 KB) + B (BN x 128 B)
     uint32_t a_bytes;
     uint32_t off_stages;    // 1024-aligned
-    uint32_t off_sf;        // LHS-scale ring: sf_stages x MW x 128 floats
-    uint32_t sf_slot_bytes;
     uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
     uint32_t sb_pitch;      // floats per sb row in smem (nkb rounded up to 4)
+    uint32_t off_out;       // output staging: one 2 KB buffer per epilogue warp
     uint32_t off_prefix;    // masked: (G + 1) ints of per-group tile prefix sums
     uint32_t off_bars;      // all mbarriers
     uint32_t off_misc;      // tmem base address, abort flag
@@ -53,8 +54,9 @@ struct Params {
     int n_blocks;   // ceil(N / BLOCK_N)
     int num_tiles;  // dense / contiguous; masked tiles are counted on the device
     int stages;
-    int sf_stages;
     SmemPlan plan;
+    const float *sa; // LHS scales, [G * K/128][ld_sa]
+    int ld_sa;
     const float *sb;
     const int *m_indices;
     const int *masked_m;
@@ -69,26 +71,25 @@ __host__ __device__ inline uint32_t align_up_u32(uint32_t x, uint32_t a)
 }
 
 // Shared-memory layout for a (MW, BN) kernel with the given ring depths.
-__host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, int sf_stages,
-                                                   int nkb, int prefix_ints)
+__host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, int nkb,
+                                                   int prefix_ints)
 {
     SmemPlan p;
     p.a_bytes = (uint32_t)mw * HALF_M * BLOCK_K;
     p.stage_bytes = p.a_bytes + (uint32_t)bn * BLOCK_K;
     p.off_stages = 0;
     uint32_t off = p.stage_bytes * (uint32_t)stages;
-    p.off_sf = align_up_u32(off, 128);
-    p.sf_slot_bytes = (uint32_t)mw * HALF_M * 4;
-    off = p.off_sf + p.sf_slot_bytes * (uint32_t)sf_stages;
     p.sb_pitch = align_up_u32((uint32_t)nkb, 4);
     p.off_sb = align_up_u32(off, 128);
     off = p.off_sb + 2u * MAX_SB_BLOCKS * p.sb_pitch * 4u;
+    p.off_out = align_up_u32(off, 1024);
+    off = p.off_out + NUM_EPI_WARPS * OUT_STAGE_BYTES;
     p.off_prefix = align_up_u32(off, 16);
     off = p.off_prefix + 4u * (uint32_t)prefix_ints;
     p.off_bars = align_up_u32(off, 8);
-    // full/empty per stage, full/empty per sf stage, tmem full/empty x2,
-    // sb full/empty x2, one "all MMAs done" barrier
-    off = p.off_bars + 8u * (2u * stages + 2u * sf_stages + 4u + 4u + 1u);
+    // full/empty per stage, TMEM full/empty per partial buffer, sb
+    // full/empty x2, one "all MMAs done" barrier
+    off = p.off_bars + 8u * (2u * stages + 2u * MAX_TMEM_BUFS + 4u + 1u);
     p.off_misc = align_up_u32(off, 16);
     p.total = p.off_misc + 16;
     return p;

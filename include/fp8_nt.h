@@ -133,7 +133,6 @@ typedef struct dg_config {
     int block_m;    /* rows per CTA tile: 128 or 256 (two 128-row MMAs) */
     int block_n;    /* columns per CTA tile: a multiple of 16 in [16, 256] */
     int stages;     /* depth of the shared-memory operand ring */
-    int sf_stages;  /* depth of the LHS-scale ring */
     int num_tiles;  /* tiles to compute (upper bound for the masked form) */
     int grid;       /* persistent CTAs launched */
     int smem_bytes; /* dynamic shared memory per CTA */

@@ -61,6 +61,20 @@ def test_dense_every_kernel_shape_ragged(mw, bn):
     H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense mw{mw} bn{bn}")
 
 
+@pytest.mark.parametrize("mw,bn", [(1, 16), (1, 32), (1, 48), (1, 64), (2, 32), (2, 64)])
+def test_dense_grouped_promotion_partial_steps(mw, bn):
+    """K = 11 blocks: promotion steps of several K blocks end with a partial step."""
+    prob = inputs.make_dense(200, 136, 128 * 11, seed=200 + bn + mw)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
+    fp8.force_config(128 * mw, bn)
+    try:
+        d = H.run_dense(prob)
+    finally:
+        fp8.force_config(0, 0)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense K=1408 mw{mw} bn{bn}")
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 8, 128), (1, 16, 128), (5, 24, 256), (128, 128, 512),
                                    (129, 136, 384), (257, 8, 128), (64, 2112, 7168)])
 def test_dense_auto_config(M, N, K):

@@ -119,7 +119,7 @@ def test_selector_invariants_and_determinism(lib):
         assert a == b
         assert a["block_m"] in (128, 256) and a["block_n"] % 16 == 0
         assert 16 <= a["block_n"] <= 256 and (a["block_m"] == 128 or a["block_n"] <= 128)
-        assert a["stages"] >= 2 and a["sf_stages"] >= a["stages"]
+        assert a["stages"] >= 2
         assert a["smem_bytes"] <= 232448
         assert a["tmem_cols"] >= 2 * (a["block_m"] // 128) * a["block_n"]
         assert a["tmem_cols"] <= 512 and a["tmem_cols"] & (a["tmem_cols"] - 1) == 0
