@@ -55,7 +55,8 @@ class DgConfig(ctypes.Structure):
     _fields_ = [("block_m", ctypes.c_int), ("block_n", ctypes.c_int),
                 ("stages", ctypes.c_int),
                 ("num_tiles", ctypes.c_int), ("grid", ctypes.c_int),
-                ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int)]
+                ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int),
+                ("split", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -88,7 +89,7 @@ def load_library():
         lib.dg_status_string.restype = ctypes.c_char_p
         lib.dg_get_device_status.argtypes = [P]
         lib.dg_select_config.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(DgConfig)]
-        lib.dg_force_config.argtypes = [I, I]
+        lib.dg_force_config.argtypes = [I, I, I]
         _lib = lib
         return lib
 
@@ -234,6 +235,8 @@ def select_config(kind: int, M: int, N: int, K: int, num_groups: int = 1,
     return cfg.as_dict()
 
 
-def force_config(block_m: int = 0, block_n: int = 0) -> None:
-    """Pin the tile shape for later calls (0, 0 = automatic).  For tests."""
-    _check(load_library().dg_force_config(int(block_m), int(block_n)), "dg_force_config")
+def force_config(block_m: int = 0, block_n: int = 0, split: int = 0) -> None:
+    """Pin the tile shape (0, 0 = automatic) and split-K factor (0 = automatic)
+    for later calls.  For tests."""
+    _check(load_library().dg_force_config(int(block_m), int(block_n), int(split)),
+           "dg_force_config")

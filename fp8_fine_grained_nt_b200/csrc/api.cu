@@ -36,6 +36,7 @@ constexpr int kDefaultSms = 148;           // B200
 constexpr int kDefaultMaxSmem = 232448;    // 227 KB opt-in per block on sm_100
 constexpr int kMaxStages = 12;
 constexpr int kMinStages = 2;
+constexpr int kMaxSplit = 4;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull; // 2 s per pipeline wait
 
 // ------------------------------------------------------------------ devices
@@ -58,7 +59,7 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
 int g_num_sms_limit = 0;
-int g_forced_bm = 0, g_forced_bn = 0;
+int g_forced_bm = 0, g_forced_bn = 0, g_forced_split = 0;
 uint64_t g_timeout_ns = 0;
 
 int device_info(DeviceInfo **out)
@@ -151,11 +152,13 @@ struct Problem {
     int expected_m; // masked only
 };
 
-// Rough cycle estimate of a (MW, BN) choice on `sms` SMs: whole waves of
-// tiles, each tile nkb K blocks long, a K block limited by the tensor pipe
-// (2 * BN cycles per 128-row MMA group at 8192 FP8 MAC/clk), operand delivery
-// (~64 B/clk/SM from L2) or the promotion FMAs (BN cycles per 128 rows).
-double estimate_cycles(const Problem &pb, int mw, int bn, int sms, int *tiles_out)
+// Rough cycle estimate of a (MW, BN, split) choice on `sms` SMs: whole
+// waves of CTAs, each working through its K blocks, a K block limited by the
+// tensor pipe (one kind::f8f6f4 MMA issues every max(64, BN/2) cycles, four
+// per 128-row block at K=32), operand delivery (~64 B/clk/SM from L2) or the
+// promotion FMAs (BN cycles per 128 rows), plus a fixed per-block pipeline
+// latency; split-K adds the cluster reduction.
+double estimate_cycles(const Problem &pb, int mw, int bn, int split, int sms, int *tiles_out)
 {
     const int bm = 128 * mw;
     const int nkb = pb.K / 128;
@@ -173,26 +176,31 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int sms, int *tiles_ou
     }
     const long n_blocks = ceil_div(pb.N, bn);
     const long tiles = m_blocks * n_blocks;
-    const long waves = (tiles + sms - 1) / sms;
+    const long ctas = tiles * split;
+    const long waves = (ctas + sms - 1) / sms;
     const int halves = (mw == 2 && rows_eff > 128) ? 2 : 1;
-    const double mma = 2.0 * bn * halves;
+    const double mma = 4.0 * halves * (bn / 2 > 64 ? bn / 2 : 64);
     const double l2 = (double)(rows_eff + bn) * 128.0 / 64.0;
     const double epi = (double)bn * halves;
     double per_kb = mma > l2 ? mma : l2;
     per_kb = per_kb > epi ? per_kb : epi;
-    per_kb += 40.0;
-    const double tile = nkb * per_kb + 1000.0;
+    per_kb += 250.0;
+    const int kb_per_cta = ceil_div(nkb, split);
+    double tile = kb_per_cta * per_kb + 1500.0;
+    if (split > 1)
+        tile += 800.0 + (double)bm * bn * 4.0 * split / 256.0 / split;
     if (tiles_out)
         *tiles_out = (int)(tiles > 0x7fffffff ? 0x7fffffff : tiles);
     return waves * tile;
 }
 
-int plan_for(const Problem &pb, int mw, int bn, int max_smem, int *stages, SmemPlan *plan)
+int plan_for(const Problem &pb, int mw, int bn, int split, int max_smem, int *stages,
+             SmemPlan *plan)
 {
     const int nkb = pb.K / 128;
     const int prefix_ints = pb.kind == DG_KIND_MASKED ? 2 * pb.groups + 1 : 0;
     for (int s = kMaxStages; s >= kMinStages; --s) {
-        SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints);
+        SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints, split > 1);
         if ((int)p.total + 1024 <= max_smem) {
             *stages = s;
             *plan = p;
@@ -202,35 +210,64 @@ int plan_for(const Problem &pb, int mw, int bn, int max_smem, int *stages, SmemP
     return DG_ERR_UNSUPPORTED_SHAPE;
 }
 
+// Clusters of `split` CTAs that can be resident at once (conservative for a
+// 148-SM part with one CTA per SM: clusters are placed within a GPC).
+int max_resident_clusters(int split, int sms)
+{
+    if (split <= 1)
+        return sms;
+    if (split == 2)
+        return sms / 2;
+    return (sms / 4) * 4 / split - 1; // leave slack for GPCs with spare SMs
+}
+
 int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand, dg_config *cfg,
            SmemPlan *plan)
 {
     const Candidate *best = nullptr;
+    int best_split = 1;
     double best_cost = 0;
+    const int nkb = pb.K / 128;
     for (int i = 0; i < kNumCandidates; ++i) {
         const Candidate &c = kCandidates[i];
         if (g_forced_bm && (c.mw * 128 != g_forced_bm || c.bn != g_forced_bn))
             continue;
         if (pb.kind == DG_KIND_CONTIGUOUS && c.mw != 1)
             continue; // a 256-row tile could straddle two 128-aligned experts
-        int st;
-        SmemPlan p;
-        if (plan_for(pb, c.mw, c.bn, max_smem, &st, &p) != DG_OK)
-            continue;
-        const double cost = estimate_cycles(pb, c.mw, c.bn, sms, nullptr);
-        // ties: wider tile first (fewer re-reads of A), then one M half
-        const bool better = !best || cost < best_cost * (1 - 1e-9) ||
-                            (fabs(cost - best_cost) <= best_cost * 1e-9 &&
-                             (c.bn > best->bn || (c.bn == best->bn && c.mw < best->mw)));
-        if (better) {
-            best = &c;
-            best_cost = cost;
+        for (int split = 1; split <= kMaxSplit; split *= 2) {
+            if (g_forced_split && split != g_forced_split)
+                continue;
+            if (split > 1) {
+                // split-K only for dense calls too small to fill the SMs
+                if (pb.kind != DG_KIND_DENSE || nkb < 2 * split)
+                    continue;
+                const long tiles = (long)ceil_div(pb.M, c.mw * 128) * ceil_div(pb.N, c.bn);
+                if (tiles * split > sms || tiles > max_resident_clusters(split, sms))
+                    continue;
+            }
+            int st;
+            SmemPlan p;
+            if (plan_for(pb, c.mw, c.bn, split, max_smem, &st, &p) != DG_OK)
+                continue;
+            // the split-K partial tile must not crowd out the operand ring
+            if (split > 1 && (c.mw * c.bn > 128 || st < 4))
+                continue;
+            const double cost = estimate_cycles(pb, c.mw, c.bn, split, sms, nullptr);
+            // ties: wider tile first (fewer re-reads of A), then one M half, then no split
+            const bool better = !best || cost < best_cost * (1 - 1e-9) ||
+                                (fabs(cost - best_cost) <= best_cost * 1e-9 &&
+                                 (c.bn > best->bn || (c.bn == best->bn && c.mw < best->mw)));
+            if (better) {
+                best = &c;
+                best_split = split;
+                best_cost = cost;
+            }
         }
     }
     if (!best)
         return DG_ERR_UNSUPPORTED_SHAPE;
     int st;
-    plan_for(pb, best->mw, best->bn, max_smem, &st, plan);
+    plan_for(pb, best->mw, best->bn, best_split, max_smem, &st, plan);
     const int bm = best->mw * 128;
     long tiles;
     if (pb.kind == DG_KIND_MASKED)
@@ -243,11 +280,17 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     cfg->block_n = best->bn;
     cfg->stages = st;
     cfg->num_tiles = (int)tiles;
-    cfg->grid = (int)(tiles < sms ? tiles : sms);
+    cfg->split = best_split;
+    if (best_split > 1)
+        cfg->grid = (int)tiles * best_split; // one tile per cluster
+    else
+        cfg->grid = (int)(tiles < sms ? tiles : sms);
     if (cfg->grid < 1)
         cfg->grid = 1;
     cfg->smem_bytes = (int)plan->total + 1024;
-    const int need = 2 * best->mw * best->bn;
+    const int buf_cols = best->mw * best->bn;
+    const int nbuf = 512 / buf_cols < MAX_TMEM_BUFS ? 512 / buf_cols : MAX_TMEM_BUFS;
+    const int need = nbuf * buf_cols; // the kernel's ring of K-block partials
     cfg->tmem_cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
     *out_cand = best;
     return DG_OK;
@@ -322,6 +365,8 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     p.m_blocks = ceil_div(pb.M, cfg.block_m);
     p.n_blocks = ceil_div(pb.N, cfg.block_n);
     p.num_tiles = cfg.num_tiles;
+    p.split = cfg.split;
+    p.kb_chunk = ceil_div(nkb, cfg.split);
     p.stages = cfg.stages;
     p.plan = plan;
     p.sa = sa;
@@ -338,6 +383,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     args.tmap_b = &tmap_b;
     args.params = &p;
     args.grid = cfg.grid;
+    args.cluster = cfg.split;
     args.smem_bytes = cfg.smem_bytes;
     args.stream = stream;
     return cand->launch(args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
@@ -487,16 +533,20 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
     return choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);
 }
 
-int dg_force_config(int block_m, int block_n)
+int dg_force_config(int block_m, int block_n, int split)
 {
+    if (split < 0 || split > kMaxSplit || (split & (split - 1)) != 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
     if (block_m == 0 && block_n == 0) {
         g_forced_bm = g_forced_bn = 0;
+        g_forced_split = split;
         return DG_OK;
     }
     for (int i = 0; i < kNumCandidates; ++i)
         if (kCandidates[i].mw * 128 == block_m && kCandidates[i].bn == block_n) {
             g_forced_bm = block_m;
             g_forced_bn = block_n;
+            g_forced_split = split;
             return DG_OK;
         }
     return DG_ERR_UNSUPPORTED_SHAPE;

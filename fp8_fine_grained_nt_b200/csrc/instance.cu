@@ -24,9 +24,22 @@ cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN)(const LaunchArgs &args)
                                            args.smem_bytes);
     if (err != cudaSuccess)
         return err;
-    kernel<<<args.grid, NUM_THREADS, args.smem_bytes, args.stream>>>(*args.tmap_a, *args.tmap_b,
-                                                                     *args.params);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)args.grid, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)args.smem_bytes;
+    cfg.stream = args.stream;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (args.cluster > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)args.cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, *args.tmap_a, *args.tmap_b, *args.params);
 }
 
 } // namespace fp8nt

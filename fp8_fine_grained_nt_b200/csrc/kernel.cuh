@@ -371,13 +371,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     const int num_tiles = (p.kind == KIND_MASKED) ? prefix[p.num_groups] : p.num_tiles;
+    // Split-K: the p.split CTAs of a cluster share one output tile, each
+    // computing K blocks [kb_lo, kb_hi); otherwise CTAs are persistent over
+    // tiles and cover all K blocks.
+    const bool split_k = p.split > 1;
+    const int split_rank = split_k ? (int)cluster_ctarank() : 0;
+    const int t_first = split_k ? (int)blockIdx.x / p.split : (int)blockIdx.x;
+    const int t_stride = split_k ? num_tiles : (int)gridDim.x;
+    const int kb_lo = split_k ? min(p.nkb, split_rank * p.kb_chunk) : 0;
+    const int kb_hi = split_k ? min(p.nkb, kb_lo + p.kb_chunk) : p.nkb;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         regs_dec<REGS_PRODUCER>();
         uint32_t stage_it = 0, tile_it = 0;
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        for (int t = t_first; ok && t < num_tiles; t += t_stride) {
             const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
             if (!ti.valid)
                 continue;
@@ -402,7 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const CUtensorMap *my_map = lane == 0 ? &tmap_b : &tmap_a;
             const int my_row = lane == 0 ? ti.b_row0 : ti.a_row0 + (lane - 1) * HALF_M;
             const uint32_t my_off = lane == 0 ? plan.a_bytes : (uint32_t)(lane - 1) * T::A_HALF_BYTES;
-            for (int kb = 0; kb < p.nkb; ++kb) {
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
                 const int s = (int)(stage_it % (uint32_t)stages);
                 int got = 1;
                 if (lane == 0) {
@@ -436,12 +445,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             constexpr uint32_t idesc = make_idesc(BN);
             uint32_t stage_it = 0, kb_it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+            for (int t = t_first; ok && t < num_tiles; t += t_stride) {
                 const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
                 if (!ti.valid)
                     continue;
                 const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
-                for (int kb = 0; kb < p.nkb; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     const int s = (int)(stage_it % (uint32_t)stages);
                     if (!wait_bar(&full[s], (stage_it / stages) & 1, abort_flag, p)) {
                         ok = false;
@@ -452,10 +461,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     // together, each warp in order: at the first block of a
                     // group, waiting for the release of the group's last
                     // buffer covers the whole group.
-                    const int gpos = kb % T::GROUP;
+                    const int gpos = (kb - kb_lo) % T::GROUP;
                     const int buf = (int)(kb_it % T::NBUF);
                     if (gpos == 0) {
-                        const int cnt = min(T::GROUP, p.nkb - kb);
+                        const int cnt = min(T::GROUP, kb_hi - kb);
                         const uint32_t last = kb_it + (uint32_t)(cnt - 1);
                         if (!wait_bar(&tmem_empty[last % T::NBUF], ((last / T::NBUF) & 1) ^ 1,
                                       abort_flag, p)) {
@@ -501,7 +510,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         uint32_t kb_it = 0, tile_it = 0;
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        for (int t = t_first; ok && t < num_tiles; t += t_stride) {
             const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
             if (!ti.valid)
                 continue;
@@ -524,9 +533,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float *sa_ptr = p.sa + (size_t)ti.sa_y0 * p.ld_sa + sa_row;
             const bool sa_ok = sa_row < p.ld_sa;
             auto sa_load = [&](int kb) {
-                return (sa_ok && kb < p.nkb) ? __ldg(sa_ptr + (size_t)kb * p.ld_sa) : 0.0f;
+                return (sa_ok && kb < kb_hi) ? __ldg(sa_ptr + (size_t)kb * p.ld_sa) : 0.0f;
             };
-            float sa_q0 = sa_load(0), sa_q1 = sa_load(1), sa_q2 = sa_load(2), sa_q3 = sa_load(3);
+            float sa_q0 = sa_load(kb_lo), sa_q1 = sa_load(kb_lo + 1), sa_q2 = sa_load(kb_lo + 2),
+                  sa_q3 = sa_load(kb_lo + 3);
             auto scales = [&](int kb, float &s_lo, float &s_hi) {
                 const float sa_v = sa_q0;
                 sa_q0 = sa_q1;
@@ -579,11 +589,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 };
                 // cur holds K blocks [kb0, kb0 + cnt), loaded and waited
                 auto step = [&](float (&cur)[64], float (&nxt)[64], int kb0) {
-                    const int cnt = min(G, p.nkb - kb0);
+                    const int cnt = min(G, kb_hi - kb0);
                     release(kb_it, cnt);
                     const int nkb0 = kb0 + cnt;
-                    const bool more = nkb0 < p.nkb;
-                    if (more && !load_step(kb_it + cnt, min(G, p.nkb - nkb0), nxt))
+                    const bool more = nkb0 < kb_hi;
+                    if (more && !load_step(kb_it + cnt, min(G, kb_hi - nkb0), nxt))
                         return false;
 #pragma unroll
                     for (int j = 0; j < G; ++j) {
@@ -603,17 +613,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     kb_it += cnt;
                     return true;
                 };
-                if (!load_step(kb_it, min(G, p.nkb), ra)) {
+                if (kb_lo >= kb_hi) {
+                    // empty K range (split-K with more splits than blocks): zero partial
+                } else if (!load_step(kb_it, min(G, kb_hi - kb_lo), ra)) {
                     ok = false;
                 } else {
                     if (active)
                         tmem_wait64(ra);
-                    for (int kb0 = 0; kb0 < p.nkb; kb0 += 2 * G) {
+                    for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += 2 * G) {
                         if (!step(ra, rb, kb0)) {
                             ok = false;
                             break;
                         }
-                        if (kb0 + G < p.nkb && !step(rb, ra, kb0 + G)) {
+                        if (kb0 + G < kb_hi && !step(rb, ra, kb0 + G)) {
                             ok = false;
                             break;
                         }
@@ -624,7 +636,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 constexpr int B0 = 64;
                 constexpr int B1 = NC - 64;
                 float r[64];
-                for (int kb = 0; kb < p.nkb; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait_full(kb_it)) {
                         ok = false;
                         break;
@@ -651,6 +663,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0)
                 mbar_arrive(&sb_empty[slot]);
             ++tile_it;
+
+            if (split_k) {
+                // split-K: leave this CTA's FP32 partial in shared memory for
+                // the cluster reduction below
+                float *red = reinterpret_cast<float *>(smem + plan.off_red);
+                float *rrow = red + row_in_tile * (BN + RED_PAD) + col0;
+#pragma unroll
+                for (int c = 0; c < NC; c += 4)
+                    *reinterpret_cast<float4 *>(rrow + c) =
+                        make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                continue;
+            }
 
             // ---- store the tile's rows as BF16
             bool row_ok = active && row_in_tile < ti.rows;
@@ -700,6 +724,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 
     __syncwarp();
+    if (split_k) {
+        // Every CTA of the cluster has its partial in shared memory; CTA r
+        // sums rows [r, r + BLOCK_M / split) of all partials in rank order
+        // (deterministic) through distributed shared memory and stores them.
+        cluster_sync();
+        const TileInfo ti = get_tile<MW, BN>(p, t_first, prefix);
+        const int rows_per = T::BLOCK_M / p.split;
+        const int r0 = split_rank * rows_per;
+        constexpr int CHUNKS = BN / 8;
+        const uint32_t red_local = smem_addr(smem + plan.off_red);
+        for (int item = threadIdx.x; item < rows_per * CHUNKS; item += NUM_THREADS) {
+            const int row = r0 + item / CHUNKS;
+            const int c8 = (item % CHUNKS) * 8;
+            if (!ti.valid || row >= ti.rows || ti.n0 + c8 >= p.N)
+                continue;
+            const uint32_t off = (uint32_t)(row * (BN + RED_PAD) + c8) * 4u;
+            float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int q = 0; q < p.split; ++q) {
+                const uint32_t remote = map_shared_rank(red_local + off, (uint32_t)q);
+                const float4 lo4 = ld_shared_cluster_v4(remote);
+                const float4 hi4 = ld_shared_cluster_v4(remote + 16);
+                s[0] += lo4.x; s[1] += lo4.y; s[2] += lo4.z; s[3] += lo4.w;
+                s[4] += hi4.x; s[5] += hi4.y; s[6] += hi4.z; s[7] += hi4.w;
+            }
+            st_global_v4(p.D + (size_t)(ti.d_row0 + row) * p.N + ti.n0 + c8, pack_bf16x2(s[0], s[1]),
+                         pack_bf16x2(s[2], s[3]), pack_bf16x2(s[4], s[5]), pack_bf16x2(s[6], s[7]));
+        }
+        // no CTA may leave (or reuse its buffer) while a peer still reads it
+        cluster_sync();
+    }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();

@@ -14,6 +14,7 @@ struct LaunchArgs {
     const CUtensorMap *tmap_b;
     const Params *params;
     int grid;
+    int cluster; // CTAs per cluster (split-K), 1 = no cluster
     int smem_bytes;
     cudaStream_t stream;
 };

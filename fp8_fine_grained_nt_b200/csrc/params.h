@@ -18,6 +18,8 @@ constexpr int MAX_SB_BLOCKS = 3;      // a BLOCK_N <= 256 tile spans at most 3 s
 constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int MAX_TMEM_BUFS = 16;      // K-block partial buffers in TMEM (ring)
 constexpr uint32_t OUT_STAGE_BYTES = 2048; // 32 rows x 32 BF16 columns per epilogue warp
+constexpr int RED_PAD = 4;             // FP32 padding per row of the split-K partial tile
+constexpr int MAX_SPLIT = 8;           // split-K CTAs per cluster (portable cluster size)
 constexpr int REGS_PRODUCER = 56;     // per-thread registers after setmaxnreg
 constexpr int REGS_EPILOGUE = 224;
 constexpr int REGS_AT_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
@@ -36,6 +38,7 @@ struct SmemPlan {
     uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
     uint32_t sb_pitch;      // floats per sb row in smem (nkb rounded up to 4)
     uint32_t off_out;       // output staging: one 2 KB buffer per epilogue warp
+    uint32_t off_red;       // split-K: this CTA's FP32 partial tile, rows padded by RED_PAD
     uint32_t off_prefix;    // masked: (G + 1) ints of per-group tile prefix sums
     uint32_t off_bars;      // all mbarriers
     uint32_t off_misc;      // tmem base address, abort flag
@@ -53,6 +56,8 @@ struct Params {
     int m_blocks;   // dense / contiguous: ceil(M / BLOCK_M); masked: per-group maximum
     int n_blocks;   // ceil(N / BLOCK_N)
     int num_tiles;  // dense / contiguous; masked tiles are counted on the device
+    int split;      // split-K CTAs per cluster (1 = off)
+    int kb_chunk;   // K blocks per split-K CTA
     int stages;
     SmemPlan plan;
     const float *sa; // LHS scales, [G * K/128][ld_sa]
@@ -72,7 +77,7 @@ __host__ __device__ inline uint32_t align_up_u32(uint32_t x, uint32_t a)
 
 // Shared-memory layout for a (MW, BN) kernel with the given ring depths.
 __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, int nkb,
-                                                   int prefix_ints)
+                                                   int prefix_ints, bool split_k)
 {
     SmemPlan p;
     p.a_bytes = (uint32_t)mw * HALF_M * BLOCK_K;
@@ -84,6 +89,9 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     off = p.off_sb + 2u * MAX_SB_BLOCKS * p.sb_pitch * 4u;
     p.off_out = align_up_u32(off, 1024);
     off = p.off_out + NUM_EPI_WARPS * OUT_STAGE_BYTES;
+    p.off_red = align_up_u32(off, 128);
+    if (split_k)
+        off = p.off_red + (uint32_t)mw * HALF_M * (uint32_t)(bn + RED_PAD) * 4u;
     p.off_prefix = align_up_u32(off, 16);
     off = p.off_prefix + 4u * (uint32_t)prefix_ints;
     p.off_bars = align_up_u32(off, 8);

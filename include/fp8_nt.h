@@ -137,6 +137,7 @@ typedef struct dg_config {
     int grid;       /* persistent CTAs launched */
     int smem_bytes; /* dynamic shared memory per CTA */
     int tmem_cols;  /* tensor-memory columns allocated per CTA */
+    int split;      /* split-K: CTAs (one thread-block cluster) sharing a tile; 1 = none */
 } dg_config;
 
 enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2 };
@@ -152,10 +153,12 @@ enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2 };
 int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected_m,
                      int num_sms, dg_config *out);
 
-/* Test hook: pin block_m / block_n for later calls (0, 0 restores automatic
- * choice).  Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is
- * built. */
-int dg_force_config(int block_m, int block_n);
+/* Test hook: pin block_m / block_n and the split-K factor for later calls
+ * (0, 0 restores automatic tile choice; split 0 = automatic, 1 = no split,
+ * 2 or 4 = that many CTAs per tile, used only where split-K applies).
+ * Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is built or the
+ * split is not 0, 1, 2 or 4. */
+int dg_force_config(int block_m, int block_n, int split);
 
 #ifdef __cplusplus
 }

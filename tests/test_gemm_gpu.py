@@ -75,6 +75,24 @@ def test_dense_grouped_promotion_partial_steps(mw, bn):
     H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense K=1408 mw{mw} bn{bn}")
 
 
+@pytest.mark.parametrize("mw,bn,split", [(1, 16, 2), (1, 64, 4), (1, 128, 2), (1, 112, 4),
+                                         (2, 32, 2), (1, 96, 4)])
+def test_dense_split_k(mw, bn, split):
+    """Split-K over a thread-block cluster: ragged M and N, K blocks not a
+    multiple of the split, reduction through distributed shared memory."""
+    prob = inputs.make_dense(100 if mw == 1 else 300, 336, 128 * 11, seed=300 + bn + split)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
+    fp8.force_config(128 * mw, bn, split)
+    try:
+        d1 = H.run_dense(prob)
+        d2 = H.run_dense(prob)
+    finally:
+        fp8.force_config(0, 0, 0)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d1), ref, f"split-K mw{mw} bn{bn} s{split}")
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16)), "split-K not deterministic"
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 8, 128), (1, 16, 128), (5, 24, 256), (128, 128, 512),
                                    (129, 136, 384), (257, 8, 128), (64, 2112, 7168)])
 def test_dense_auto_config(M, N, K):

@@ -128,6 +128,27 @@ def test_selector_invariants_and_determinism(lib):
             assert a["block_m"] == 128
 
 
+def test_decode_shape_uses_split_k_in_one_wave(lib):
+    cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)
+    assert cfg["split"] in (2, 4)
+    assert cfg["grid"] == cfg["num_tiles"] * cfg["split"] <= 148
+    # large problems never split
+    assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["split"] == 1
+    assert fp8.select_config(fp8.KIND_CONTIGUOUS, 128 * 40, 4096, 7168, 8, num_sms=148)["split"] == 1
+    assert fp8.select_config(fp8.KIND_MASKED, 256, 4096, 7168, 16, num_sms=148)["split"] == 1
+
+
+def test_forced_split(lib):
+    try:
+        fp8.force_config(128, 64, 4)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)
+        assert (cfg["block_n"], cfg["split"]) == (64, 4)
+        with pytest.raises(fp8.Fp8NtError):
+            fp8.force_config(128, 64, 3)
+    finally:
+        fp8.force_config(0, 0, 0)
+
+
 def test_force_config_rejects_unbuilt_shapes(lib):
     with pytest.raises(fp8.Fp8NtError):
         fp8.force_config(128, 120)
