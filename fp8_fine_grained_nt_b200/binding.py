@@ -56,7 +56,7 @@ class DgConfig(ctypes.Structure):
                 ("stages", ctypes.c_int),
                 ("num_tiles", ctypes.c_int), ("grid", ctypes.c_int),
                 ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int),
-                ("split", ctypes.c_int)]
+                ("split", ctypes.c_int), ("cta_pair", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -89,7 +89,7 @@ def load_library():
         lib.dg_status_string.restype = ctypes.c_char_p
         lib.dg_get_device_status.argtypes = [P]
         lib.dg_select_config.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(DgConfig)]
-        lib.dg_force_config.argtypes = [I, I, I]
+        lib.dg_force_config.argtypes = [I, I, I, I]
         _lib = lib
         return lib
 
@@ -235,8 +235,9 @@ def select_config(kind: int, M: int, N: int, K: int, num_groups: int = 1,
     return cfg.as_dict()
 
 
-def force_config(block_m: int = 0, block_n: int = 0, split: int = 0) -> None:
-    """Pin the tile shape (0, 0 = automatic) and split-K factor (0 = automatic)
+def force_config(block_m: int = 0, block_n: int = 0, split: int = 0, cta_pair: int = 0) -> None:
+    """Pin the tile shape (0, 0 = automatic), split-K factor (0 = automatic)
+    and CTA-pair mode (0 = automatic, 1 = one CTA per tile, 2 = CTA pairs)
     for later calls.  For tests."""
-    _check(load_library().dg_force_config(int(block_m), int(block_n), int(split)),
-           "dg_force_config")
+    _check(load_library().dg_force_config(int(block_m), int(block_n), int(split),
+                                          int(cta_pair)), "dg_force_config")

@@ -22,11 +22,12 @@ namespace {
 struct Candidate {
     int mw;
     int bn;
+    int pair; // 1: a CTA pair computes a 256-row tile (tcgen05 cta_group::2)
     LaunchFn launch;
 };
 
 const Candidate kCandidates[] = {
-#define FP8NT_KERNEL(mw, bn) {mw, bn, launch_mw##mw##_bn##bn},
+#define FP8NT_KERNEL(mw, bn, pair) {mw, bn, pair, launch_mw##mw##_bn##bn##_p##pair},
 #include "kernels.def"
 #undef FP8NT_KERNEL
 };
@@ -59,7 +60,7 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
 int g_num_sms_limit = 0;
-int g_forced_bm = 0, g_forced_bn = 0, g_forced_split = 0;
+int g_forced_bm = 0, g_forced_bn = 0, g_forced_split = 0, g_forced_pair = 0;
 uint64_t g_timeout_ns = 0;
 
 int device_info(DeviceInfo **out)
@@ -152,15 +153,17 @@ struct Problem {
     int expected_m; // masked only
 };
 
-// Rough cycle estimate of a (MW, BN, split) choice on `sms` SMs: whole
+// Rough cycle estimate of a (MW, BN, split, pair) choice on `sms` SMs: whole
 // waves of CTAs, each working through its K blocks, a K block limited by the
 // tensor pipe (one kind::f8f6f4 MMA issues every max(64, BN/2) cycles, four
-// per 128-row block at K=32), operand delivery (~64 B/clk/SM from L2) or the
-// promotion FMAs (BN cycles per 128 rows), plus a fixed per-block pipeline
-// latency; split-K adds the cluster reduction.
-double estimate_cycles(const Problem &pb, int mw, int bn, int split, int sms, int *tiles_out)
+// per 128-row block at K=32), operand delivery (~64 B/clk/SM from L2; a CTA
+// of a pair loads half of B) or the promotion FMAs (BN cycles per 128 rows),
+// plus a fixed per-block pipeline latency; split-K adds the cluster
+// reduction.
+double estimate_cycles(const Problem &pb, int mw, int bn, int split, int pair, int stages, int sms,
+                       int *tiles_out)
 {
-    const int bm = 128 * mw;
+    const int bm = pair ? 256 : 128 * mw;
     const int nkb = pb.K / 128;
     long m_blocks;
     int rows_eff;
@@ -176,12 +179,14 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int split, int sms, in
     }
     const long n_blocks = ceil_div(pb.N, bn);
     const long tiles = m_blocks * n_blocks;
-    const long ctas = tiles * split;
+    const long ctas = tiles * split * (pair ? 2 : 1);
     const long waves = (ctas + sms - 1) / sms;
     const int halves = (mw == 2 && rows_eff > 128) ? 2 : 1;
     const double mma = 4.0 * halves * (bn / 2 > 64 ? bn / 2 : 64);
-    const double l2 = (double)(rows_eff + bn) * 128.0 / 64.0;
+    const int a_rows = pair ? 128 : rows_eff;
+    const double l2 = (double)(a_rows + (pair ? bn / 2 : bn)) * 128.0 / 64.0;
     const double epi = (double)bn * halves;
+    (void)stages;
     double per_kb = mma > l2 ? mma : l2;
     per_kb = per_kb > epi ? per_kb : epi;
     per_kb += 250.0;
@@ -194,13 +199,13 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int split, int sms, in
     return waves * tile;
 }
 
-int plan_for(const Problem &pb, int mw, int bn, int split, int max_smem, int *stages,
+int plan_for(const Problem &pb, int mw, int bn, int split, int pair, int max_smem, int *stages,
              SmemPlan *plan)
 {
     const int nkb = pb.K / 128;
     const int prefix_ints = pb.kind == DG_KIND_MASKED ? 2 * pb.groups + 1 : 0;
     for (int s = kMaxStages; s >= kMinStages; --s) {
-        SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints, split > 1);
+        SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints, split > 1, pair != 0);
         if ((int)p.total + 1024 <= max_smem) {
             *stages = s;
             *plan = p;
@@ -230,12 +235,21 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     const int nkb = pb.K / 128;
     for (int i = 0; i < kNumCandidates; ++i) {
         const Candidate &c = kCandidates[i];
-        if (g_forced_bm && (c.mw * 128 != g_forced_bm || c.bn != g_forced_bn))
+        const int c_bm = c.pair ? 256 : c.mw * 128;
+        if (g_forced_bm && (c_bm != g_forced_bm || c.bn != g_forced_bn))
             continue;
-        if (pb.kind == DG_KIND_CONTIGUOUS && c.mw != 1)
+        if (g_forced_pair && (g_forced_pair == 2) != (c.pair != 0))
+            continue;
+        // CTA pairs only on request: measured on B200 they were no faster
+        // than one CTA per tile on the dense, masked and 256-row shapes
+        if (c.pair && g_forced_pair != 2)
+            continue;
+        if (pb.kind == DG_KIND_CONTIGUOUS && c_bm != 128)
             continue; // a 256-row tile could straddle two 128-aligned experts
         for (int split = 1; split <= kMaxSplit; split *= 2) {
             if (g_forced_split && split != g_forced_split)
+                continue;
+            if (c.pair && split > 1)
                 continue;
             if (split > 1) {
                 // split-K only for dense calls too small to fill the SMs
@@ -247,16 +261,20 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
             }
             int st;
             SmemPlan p;
-            if (plan_for(pb, c.mw, c.bn, split, max_smem, &st, &p) != DG_OK)
+            if (plan_for(pb, c.mw, c.bn, split, c.pair, max_smem, &st, &p) != DG_OK)
                 continue;
             // the split-K partial tile must not crowd out the operand ring
             if (split > 1 && (c.mw * c.bn > 128 || st < 4))
                 continue;
-            const double cost = estimate_cycles(pb, c.mw, c.bn, split, sms, nullptr);
-            // ties: wider tile first (fewer re-reads of A), then one M half, then no split
-            const bool better = !best || cost < best_cost * (1 - 1e-9) ||
-                                (fabs(cost - best_cost) <= best_cost * 1e-9 &&
-                                 (c.bn > best->bn || (c.bn == best->bn && c.mw < best->mw)));
+            const double cost = estimate_cycles(pb, c.mw, c.bn, split, c.pair, st, sms, nullptr);
+            // ties: wider tile first (fewer re-reads of A), then one M half,
+            // then a single CTA, then no split
+            const bool better =
+                !best || cost < best_cost * (1 - 1e-9) ||
+                (fabs(cost - best_cost) <= best_cost * 1e-9 &&
+                 (c.bn > best->bn ||
+                  (c.bn == best->bn &&
+                   (c.mw < best->mw || (c.mw == best->mw && c.pair < best->pair)))));
             if (better) {
                 best = &c;
                 best_split = split;
@@ -267,8 +285,8 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     if (!best)
         return DG_ERR_UNSUPPORTED_SHAPE;
     int st;
-    plan_for(pb, best->mw, best->bn, best_split, max_smem, &st, plan);
-    const int bm = best->mw * 128;
+    plan_for(pb, best->mw, best->bn, best_split, best->pair, max_smem, &st, plan);
+    const int bm = best->pair ? 256 : best->mw * 128;
     long tiles;
     if (pb.kind == DG_KIND_MASKED)
         tiles = (long)pb.groups * ceil_div(pb.M, bm) * ceil_div(pb.N, best->bn);
@@ -281,8 +299,11 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     cfg->stages = st;
     cfg->num_tiles = (int)tiles;
     cfg->split = best_split;
+    cfg->cta_pair = best->pair ? 2 : 1;
     if (best_split > 1)
         cfg->grid = (int)tiles * best_split; // one tile per cluster
+    else if (best->pair)
+        cfg->grid = 2 * (int)(tiles < sms / 2 ? tiles : sms / 2); // persistent pairs
     else
         cfg->grid = (int)(tiles < sms ? tiles : sms);
     if (cfg->grid < 1)
@@ -349,8 +370,10 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, a_rows, pb.K, 128,
                            128, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
         return st;
+    // a CTA of a pair loads half of the B tile
+    const uint32_t b_box_rows = cand->pair ? cfg.block_n / 2 : cfg.block_n;
     if ((st = make_tmap_2d(&tmap_b, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, b_rows, pb.K, 128,
-                           cfg.block_n, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+                           b_box_rows, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
         return st;
 
     Params p;
@@ -383,7 +406,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     args.tmap_b = &tmap_b;
     args.params = &p;
     args.grid = cfg.grid;
-    args.cluster = cfg.split;
+    args.cluster = cand->pair ? 2 : cfg.split;
     args.smem_bytes = cfg.smem_bytes;
     args.stream = stream;
     return cand->launch(args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
@@ -533,22 +556,29 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
     return choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);
 }
 
-int dg_force_config(int block_m, int block_n, int split)
+int dg_force_config(int block_m, int block_n, int split, int cta_pair)
 {
     if (split < 0 || split > kMaxSplit || (split & (split - 1)) != 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    if (cta_pair < 0 || cta_pair > 2)
         return DG_ERR_UNSUPPORTED_SHAPE;
     if (block_m == 0 && block_n == 0) {
         g_forced_bm = g_forced_bn = 0;
         g_forced_split = split;
+        g_forced_pair = cta_pair;
         return DG_OK;
     }
-    for (int i = 0; i < kNumCandidates; ++i)
-        if (kCandidates[i].mw * 128 == block_m && kCandidates[i].bn == block_n) {
+    for (int i = 0; i < kNumCandidates; ++i) {
+        const Candidate &c = kCandidates[i];
+        if ((c.pair ? 256 : c.mw * 128) == block_m && c.bn == block_n &&
+            (cta_pair == 0 || (cta_pair == 2) == (c.pair != 0))) {
             g_forced_bm = block_m;
             g_forced_bn = block_n;
             g_forced_split = split;
+            g_forced_pair = cta_pair;
             return DG_OK;
         }
+    }
     return DG_ERR_UNSUPPORTED_SHAPE;
 }
 

@@ -1,5 +1,6 @@
-// One (MW, BN) instantiation of the GEMM kernel and its launcher; the build
-// compiles this file once per entry of kernels.def with -DFP8NT_MW / -DFP8NT_BN.
+// One (MW, BN, PAIR) instantiation of the GEMM kernel and its launcher; the
+// build compiles this file once per entry of kernels.def with -DFP8NT_MW,
+// -DFP8NT_BN and -DFP8NT_PAIR.
 #include <cuda_runtime.h>
 
 #include "kernel.cuh"
@@ -11,21 +12,54 @@
 #ifndef FP8NT_BN
 #error "FP8NT_BN must be defined"
 #endif
+#ifndef FP8NT_PAIR
+#error "FP8NT_PAIR must be defined"
+#endif
 
 namespace fp8nt {
 
-#define FP8NT_CAT_(a, b, c) launch_mw##a##_bn##b##c
-#define FP8NT_NAME(a, b) FP8NT_CAT_(a, b, )
+#define FP8NT_CAT_(a, b, c) launch_mw##a##_bn##b##_p##c
+#define FP8NT_NAME(a, b, c) FP8NT_CAT_(a, b, c)
 
-cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN)(const LaunchArgs &args)
+cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN, FP8NT_PAIR)(const LaunchArgs &args)
 {
-    auto kernel = fp8_gemm_kernel<FP8NT_MW, FP8NT_BN>;
+    auto kernel = fp8_gemm_kernel<FP8NT_MW, FP8NT_BN, FP8NT_PAIR != 0>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            args.smem_bytes);
     if (err != cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)args.grid, 1, 1);
+    int grid = args.grid;
+    if (FP8NT_PAIR && args.cluster == 2) {
+        // persistent pairs: no more than can be resident at once (a GPC with
+        // an odd number of free SMs holds one CTA fewer than a naive count)
+        static int max_pairs[64] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return cudaErrorInvalidDevice;
+        if (max_pairs[dev] == 0) {
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3((unsigned)args.grid, 1, 1);
+            q.blockDim = dim3(NUM_THREADS, 1, 1);
+            q.dynamicSmemBytes = (size_t)args.smem_bytes;
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = 2;
+            qa[0].val.clusterDim.y = 1;
+            qa[0].val.clusterDim.z = 1;
+            q.attrs = qa;
+            q.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kernel, &q) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = 1 << 30; // unknown: keep the host's choice
+            }
+            max_pairs[dev] = n;
+        }
+        if (grid > 2 * max_pairs[dev])
+            grid = 2 * max_pairs[dev];
+    }
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)args.smem_bytes;
     cfg.stream = args.stream;

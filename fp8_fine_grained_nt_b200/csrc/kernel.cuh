@@ -35,12 +35,15 @@
 
 namespace fp8nt {
 
-template <int MW, int BN>
+template <int MW, int BN, bool PAIR = false>
 struct KernelTraits {
     static_assert(MW == 1 || MW == 2, "MW is 1 or 2");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be a multiple of 16 in [16, 256]");
     static_assert(MW == 1 || BN <= 128, "two M halves need BN <= 128 (TMEM and registers)");
-    static constexpr int BLOCK_M = MW * HALF_M;
+    static_assert(!PAIR || (MW == 1 && BN % 32 == 0), "a CTA pair splits B in halves of BN/2 rows");
+    // rows of the tile a CTA (or, with PAIR, a CTA pair) computes
+    static constexpr int BLOCK_M = PAIR ? 2 * HALF_M : MW * HALF_M;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN; // rows of B each CTA loads
     static constexpr int BUF_COLS = MW * BN;                 // TMEM columns per K-block buffer
     // ring of K-block partial buffers in TMEM: as many as fit, at most 16
     static constexpr int NBUF = (512 / BUF_COLS) < MAX_TMEM_BUFS ? (512 / BUF_COLS) : MAX_TMEM_BUFS;
@@ -57,20 +60,20 @@ struct KernelTraits {
     static constexpr int GROUP_BY_REGS = PREFETCH ? 64 / COLS_PER_THREAD : 1;
     static constexpr int GROUP = GROUP_BY_REGS < NBUF / 2 ? GROUP_BY_REGS : (NBUF / 2 > 0 ? NBUF / 2 : 1);
     static constexpr uint32_t A_HALF_BYTES = HALF_M * BLOCK_K;
-    static constexpr uint32_t B_BYTES = BN * BLOCK_K;
+    static constexpr uint32_t B_BYTES = B_ROWS * BLOCK_K;
     static_assert(NBUF >= 2 && NBUF <= MAX_TMEM_BUFS && TMEM_NEED <= 512, "TMEM holds 512 columns");
     static_assert(COLS_PER_THREAD % 8 == 0, "epilogue works in 8-column chunks");
 };
 
 // Instruction descriptor of tcgen05.mma kind::f8f6f4: D FP32, A and B E4M3,
-// both K-major, M = 128, N = BN, dense.
-__host__ __device__ constexpr uint32_t make_idesc(int bn)
+// both K-major, M = 128 (256 for a CTA pair), N = BN, dense.
+__host__ __device__ constexpr uint32_t make_idesc(int bn, int m = HALF_M)
 {
     return (1u << 4)                          // D format: F32
            | (0u << 7) | (0u << 10)           // A, B format: E4M3
            | (0u << 15) | (0u << 16)          // A, B K-major
            | ((uint32_t)(bn >> 3) << 17)      // N / 8
-           | ((uint32_t)(HALF_M >> 4) << 24); // M / 16
+           | ((uint32_t)(m >> 4) << 24);      // M / 16
 }
 
 // Shared-memory matrix descriptor for a K-major tile written by TMA with the
@@ -98,10 +101,10 @@ struct TileInfo {
     int d_row0;  // row of D (all groups flattened) holding row m0
 };
 
-template <int MW, int BN>
-__device__ __forceinline__ TileInfo get_tile(const Params &p, int t, const int *prefix)
+template <int MW, int BN, bool PAIR>
+__device__ __forceinline__ TileInfo get_tile(const Params &p, int t, const int *prefix, int pair_rank)
 {
-    constexpr int BM = KernelTraits<MW, BN>::BLOCK_M;
+    constexpr int BM = KernelTraits<MW, BN, PAIR>::BLOCK_M;
     TileInfo ti;
     ti.valid = 1;
     int mb, nb;
@@ -150,6 +153,15 @@ __device__ __forceinline__ TileInfo get_tile(const Params &p, int t, const int *
                 ti.b_row0 = e * p.N + nb * BN;
             }
         }
+    }
+    if (PAIR) {
+        // this CTA's 128 rows of the pair's 256, and its half of B
+        const int off = pair_rank * HALF_M;
+        ti.m0 += off;
+        ti.a_row0 += off;
+        ti.d_row0 += off;
+        ti.rows = max(0, min(HALF_M, ti.rows - off));
+        ti.b_row0 += pair_rank * (BN / 2);
     }
     ti.n0 = nb * BN;
     const int nb128 = ti.n0 >> 7;
@@ -282,12 +294,12 @@ __device__ __forceinline__ void fma_range_any(float (&acc)[NC], const float (&v)
         fma_range<NC, C0, N, false>(acc, v, s_lo, s_hi, t);
 }
 
-template <int MW, int BN>
+template <int MW, int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ Params p)
 {
-    using T = KernelTraits<MW, BN>;
+    using T = KernelTraits<MW, BN, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -318,7 +330,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int b = 0; b < T::NBUF; ++b) {
             mbar_init(&tmem_full[b], 1);
-            mbar_init(&tmem_empty[b], NUM_EPI_WARPS);
+            // a pair's leader also counts the peer's epilogue warps
+            mbar_init(&tmem_empty[b], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sb_full[b], 32);
@@ -333,8 +346,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmap_b);
     }
     if (warp == 1) {
-        tmem_alloc(misc, T::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(misc, T::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(misc, T::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     if (p.kind == KIND_MASKED && warp == 2) {
         // Tiles per group = ceil(masked_m / BLOCK_M) * n_blocks; prefix sums
@@ -367,17 +385,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             prefix[p.num_groups] = carry;
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR)
+        cluster_sync(); // the peer may arrive on the leader's barriers from here on
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     const int num_tiles = (p.kind == KIND_MASKED) ? prefix[p.num_groups] : p.num_tiles;
     // Split-K: the p.split CTAs of a cluster share one output tile, each
     // computing K blocks [kb_lo, kb_hi); otherwise CTAs are persistent over
     // tiles and cover all K blocks.
-    const bool split_k = p.split > 1;
+    const bool split_k = !PAIR && p.split > 1;
     const int split_rank = split_k ? (int)cluster_ctarank() : 0;
-    const int t_first = split_k ? (int)blockIdx.x / p.split : (int)blockIdx.x;
-    const int t_stride = split_k ? num_tiles : (int)gridDim.x;
+    // a CTA pair walks the pair tiles together; rank 0 is the leader
+    const int pair_rank = PAIR ? (int)cluster_ctarank() : 0;
+    const bool leader = pair_rank == 0;
+    const int t_first = split_k ? (int)blockIdx.x / p.split
+                                : (PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x);
+    const int t_stride = split_k ? num_tiles : (PAIR ? (int)gridDim.x / 2 : (int)gridDim.x);
     const int kb_lo = split_k ? min(p.nkb, split_rank * p.kb_chunk) : 0;
     const int kb_hi = split_k ? min(p.nkb, kb_lo + p.kb_chunk) : p.nkb;
 
@@ -387,7 +412,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t stage_it = 0, tile_it = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-            const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
+            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
             if (!ti.valid)
                 continue;
             // RHS scales of the whole tile: <= 3 rows of K/128 floats
@@ -416,24 +441,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 int got = 1;
                 if (lane == 0) {
                     got = wait_bar(&empty[s], ((stage_it / stages) & 1) ^ 1, abort_flag, p) ? 1 : 0;
-                    if (got)
-                        mbar_arrive_expect_tx(&full[s], ab_bytes);
+                    // a pair's leader expects both CTAs' bytes on its barrier
+                    if (got && leader)
+                        mbar_arrive_expect_tx(&full[s], PAIR ? 2 * ab_bytes : ab_bytes);
                 }
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (!got) {
                     ok = false;
                     break;
                 }
-                if (copier)
-                    tma_load_2d(smem + plan.off_stages + (uint32_t)s * plan.stage_bytes + my_off,
-                                my_map, &full[s], kb * BLOCK_K, my_row);
+                if (copier) {
+                    uint8_t *dst = smem + plan.off_stages + (uint32_t)s * plan.stage_bytes + my_off;
+                    if constexpr (PAIR)
+                        tma_load_2d_pair(dst, my_map, map_shared_rank(smem_addr(&full[s]), 0u),
+                                         kb * BLOCK_K, my_row);
+                    else
+                        tma_load_2d(dst, my_map, &full[s], kb * BLOCK_K, my_row);
+                }
                 ++stage_it;
             }
             ++tile_it;
         }
         // Drain: every copy issued must land before the CTA exits.
         cp_async_wait_all();
-        if (lane == 0) {
+        if (lane == 0 && leader) { // a peer's copies are drained through the leader's barriers
             const uint32_t n = stage_it < (uint32_t)stages ? stage_it : (uint32_t)stages;
             for (uint32_t i = stage_it - n; i < stage_it; ++i)
                 wait_drain(&full[i % stages], (i / stages) & 1, abort_flag, p);
@@ -441,12 +472,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         regs_dec<REGS_PRODUCER>();
-        if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc(BN);
+        if (lane == 0 && leader) { // a pair's MMAs are issued by the leader alone
+            constexpr uint32_t idesc = make_idesc(BN, PAIR ? 2 * HALF_M : HALF_M);
             uint32_t stage_it = 0, kb_it = 0;
             bool ok = true;
             for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-                const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
+                const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
                 if (!ti.valid)
                     continue;
                 const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
@@ -479,20 +510,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int h = 0; h < halves; ++h) {
                         const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS + h * BN);
 #pragma unroll
-                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
-                            mma_f8f6f4(d, make_sdesc(a_base + h * T::A_HALF_BYTES + k * MMA_K),
-                                       make_sdesc(b_base + k * MMA_K), idesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
+                            const uint64_t ad = make_sdesc(a_base + h * T::A_HALF_BYTES + k * MMA_K);
+                            const uint64_t bd = make_sdesc(b_base + k * MMA_K);
+                            if constexpr (PAIR)
+                                mma_f8f6f4_pair(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                            else
+                                mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        }
                     }
-                    mma_commit(&empty[s]);
                     // every buffer completes one phase per use (the epilogue
-                    // waits only for a group's last one)
-                    mma_commit(&tmem_full[buf]);
+                    // waits only for a group's last one); a pair's commits
+                    // reach both CTAs
+                    if constexpr (PAIR) {
+                        mma_commit_pair_mc(&empty[s], 0x3);
+                        mma_commit_pair_mc(&tmem_full[buf], 0x3);
+                    } else {
+                        mma_commit(&empty[s]);
+                        mma_commit(&tmem_full[buf]);
+                    }
                     ++stage_it;
                     ++kb_it;
                 }
             }
             // Drain: all MMAs complete before TMEM is released.
-            mma_commit(mma_done);
+            if constexpr (PAIR)
+                mma_commit_pair(mma_done);
+            else
+                mma_commit(mma_done);
             wait_drain(mma_done, 0, abort_flag, p);
         }
     } else if (warp < FIRST_EPI_WARP) {
@@ -511,14 +556,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t kb_it = 0, tile_it = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-            const TileInfo ti = get_tile<MW, BN>(p, t, prefix);
+            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
             if (!ti.valid)
                 continue;
             const int slot = tile_it & 1;
             if (!wait_bar_warp(&sb_full[slot], (tile_it >> 1) & 1, abort_flag, p))
                 break;
             const float *sbt = sb_tile + slot * MAX_SB_BLOCKS * pitch;
-            const bool active = (MW == 1) || (half * HALF_M < ti.rows);
+            const bool active = (MW == 1) ? true : (half * HALF_M < ti.rows);
             const int cbase = ti.n0 + col0;
             // scale blocks of this thread's columns: lo = block of its first
             // column (relative to the tile's first block), t_split = local
@@ -565,8 +610,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    for (int j = 0; j < cnt; ++j)
-                        mbar_arrive(&tmem_empty[(it + j) % T::NBUF]);
+                    for (int j = 0; j < cnt; ++j) {
+                        uint64_t *bar = &tmem_empty[(it + j) % T::NBUF];
+                        if (PAIR && !leader)
+                            mbar_arrive_cluster(map_shared_rank(smem_addr(bar), 0u));
+                        else
+                            mbar_arrive(bar);
+                    }
             };
             if constexpr (T::PREFETCH) {
                 // Steps of up to GROUP K blocks: their partials are loaded
@@ -729,7 +779,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // sums rows [r, r + BLOCK_M / split) of all partials in rank order
         // (deterministic) through distributed shared memory and stores them.
         cluster_sync();
-        const TileInfo ti = get_tile<MW, BN>(p, t_first, prefix);
+        const TileInfo ti = get_tile<MW, BN, PAIR>(p, t_first, prefix, pair_rank);
         const int rows_per = T::BLOCK_M / p.split;
         const int r0 = split_rank * rows_per;
         constexpr int CHUNKS = BN / 8;
@@ -754,10 +804,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // no CTA may leave (or reuse its buffer) while a peer still reads it
         cluster_sync();
     }
-    __syncthreads();
+    if constexpr (PAIR)
+        cluster_sync(); // neither CTA leaves while its pair may still use its memory
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, T::TMEM_COLS);
+        if constexpr (PAIR)
+            tmem_dealloc_pair(tmem_base, T::TMEM_COLS);
+        else
+            tmem_dealloc(tmem_base, T::TMEM_COLS);
     }
 }
 

@@ -14,14 +14,14 @@ struct LaunchArgs {
     const CUtensorMap *tmap_b;
     const Params *params;
     int grid;
-    int cluster; // CTAs per cluster (split-K), 1 = no cluster
+    int cluster; // CTAs per cluster (split-K, or 2 for a CTA pair), 1 = no cluster
     int smem_bytes;
     cudaStream_t stream;
 };
 
 typedef cudaError_t (*LaunchFn)(const LaunchArgs &);
 
-#define FP8NT_KERNEL(mw, bn) cudaError_t launch_mw##mw##_bn##bn(const LaunchArgs &);
+#define FP8NT_KERNEL(mw, bn, pair) cudaError_t launch_mw##mw##_bn##bn##_p##pair(const LaunchArgs &);
 #include "kernels.def"
 #undef FP8NT_KERNEL
 

@@ -32,7 +32,7 @@ constexpr uint32_t DEVERR_TIMEOUT = 1u;
 constexpr uint32_t DEVERR_BAD_INDEX = 2u;
 
 struct SmemPlan {
-    uint32_t stage_bytes;   // A (MW x 16 KB) + B (BN x 128 B)
+    uint32_t stage_bytes;   // A (MW x 16 KB) + B (BN x 128 B; BN/2 rows per CTA of a pair)
     uint32_t a_bytes;
     uint32_t off_stages;    // 1024-aligned
     uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
@@ -75,13 +75,14 @@ __host__ __device__ inline uint32_t align_up_u32(uint32_t x, uint32_t a)
     return (x + a - 1) / a * a;
 }
 
-// Shared-memory layout for a (MW, BN) kernel with the given ring depths.
+// Shared-memory layout for a (MW, BN) kernel with the given ring depths; a
+// CTA of a pair holds half of the B tile.
 __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, int nkb,
-                                                   int prefix_ints, bool split_k)
+                                                   int prefix_ints, bool split_k, bool pair = false)
 {
     SmemPlan p;
     p.a_bytes = (uint32_t)mw * HALF_M * BLOCK_K;
-    p.stage_bytes = p.a_bytes + (uint32_t)bn * BLOCK_K;
+    p.stage_bytes = p.a_bytes + (uint32_t)(pair ? bn / 2 : bn) * BLOCK_K;
     p.off_stages = 0;
     uint32_t off = p.stage_bytes * (uint32_t)stages;
     p.sb_pitch = align_up_u32((uint32_t)nkb, 4);

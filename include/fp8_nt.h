@@ -130,7 +130,8 @@ int dg_get_device_status(dg_stream_t stream);
 
 /* Tile configuration chosen for a call (host logic; no GPU needed). */
 typedef struct dg_config {
-    int block_m;    /* rows per CTA tile: 128 or 256 (two 128-row MMAs) */
+    int block_m;    /* rows per tile: 128, or 256 (two 128-row MMAs in one CTA,
+                       or one 256-row MMA over a CTA pair) */
     int block_n;    /* columns per CTA tile: a multiple of 16 in [16, 256] */
     int stages;     /* depth of the shared-memory operand ring */
     int num_tiles;  /* tiles to compute (upper bound for the masked form) */
@@ -138,6 +139,9 @@ typedef struct dg_config {
     int smem_bytes; /* dynamic shared memory per CTA */
     int tmem_cols;  /* tensor-memory columns allocated per CTA */
     int split;      /* split-K: CTAs (one thread-block cluster) sharing a tile; 1 = none */
+    int cta_pair;   /* 2: a cluster of two CTAs computes each 256-row tile with
+                       tcgen05 cta_group::2 MMAs (each CTA loads its own 128 rows
+                       of A and half of the B tile); 1: one CTA per tile */
 } dg_config;
 
 enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2 };
@@ -153,12 +157,13 @@ enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2 };
 int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected_m,
                      int num_sms, dg_config *out);
 
-/* Test hook: pin block_m / block_n and the split-K factor for later calls
- * (0, 0 restores automatic tile choice; split 0 = automatic, 1 = no split,
- * 2 or 4 = that many CTAs per tile, used only where split-K applies).
- * Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is built or the
- * split is not 0, 1, 2 or 4. */
-int dg_force_config(int block_m, int block_n, int split);
+/* Test hook: pin block_m / block_n, the split-K factor and the CTA-pair mode
+ * for later calls (0, 0 restores automatic tile choice; split 0 = automatic,
+ * 1 = no split, 2 or 4 = that many CTAs per tile, used only where split-K
+ * applies; cta_pair 0 = automatic, 1 = one CTA per tile, 2 = CTA pairs).
+ * Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is built, the
+ * split is not 0, 1, 2 or 4, or cta_pair is not 0, 1 or 2. */
+int dg_force_config(int block_m, int block_n, int split, int cta_pair);
 
 #ifdef __cplusplus
 }

@@ -47,18 +47,59 @@ def check_status():
 # --------------------------------------------------------------------- dense
 
 
-@pytest.mark.parametrize("mw,bn", built_shapes())
-def test_dense_every_kernel_shape_ragged(mw, bn):
+def force_shape(mw, bn, pair, split=0):
+    """Pin one built kernel: (MW, BN) with one CTA per tile, or a CTA pair."""
+    fp8.force_config(256 if pair else 128 * mw, bn, split, 2 if pair else 1)
+
+
+@pytest.mark.parametrize("mw,bn,pair", built_shapes())
+def test_dense_every_kernel_shape_ragged(mw, bn, pair):
     """Each built tile shape on a shape with ragged M, N tails and several K blocks."""
-    prob = inputs.make_dense(300, 400, 512, seed=100 + bn + mw)
+    prob = inputs.make_dense(300, 400, 512, seed=100 + bn + mw + 7 * pair)
     ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
-    fp8.force_config(128 * mw, bn)
+    force_shape(mw, bn, pair)
     try:
+        cfg = fp8.select_config(fp8.KIND_DENSE, prob.M, prob.N, prob.K)
+        assert cfg["cta_pair"] == (2 if pair else 1)
         d = H.run_dense(prob)
     finally:
         fp8.force_config(0, 0)
     check_status()
-    H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense mw{mw} bn{bn}")
+    H.assert_close(H.bf16_bits_to_f64(d), ref, f"dense mw{mw} bn{bn} pair{pair}")
+
+
+@pytest.mark.parametrize("M", [1, 100, 128, 200, 256, 300, 520])
+@pytest.mark.parametrize("bn", [128, 256])
+def test_dense_cta_pair_row_edges(M, bn):
+    """CTA pairs where the second CTA's 128 rows are partly or wholly past M,
+    with 11 K blocks (a partial promotion step) and a ragged N tail."""
+    prob = inputs.make_dense(M, bn * 2 + 40, 128 * 11, seed=400 + M + bn)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
+    force_shape(1, bn, True)
+    try:
+        d1 = H.run_dense(prob)
+        d2 = H.run_dense(prob)
+    finally:
+        fp8.force_config(0, 0)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d1), ref, f"pair M{M} bn{bn}")
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+def test_dense_cta_pair_more_tiles_than_pairs():
+    """A pair walks several 256-row tiles (persistent loop) with the SM
+    bound lowered so that every pair takes many tiles."""
+    prob = inputs.make_dense(1000, 1040, 1024, seed=77)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
+    force_shape(1, 160, True)
+    fp8.set_num_sms(8)
+    try:
+        d = H.run_dense(prob)
+    finally:
+        fp8.set_num_sms(0)
+        fp8.force_config(0, 0)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, "pair persistent")
 
 
 @pytest.mark.parametrize("mw,bn", [(1, 16), (1, 32), (1, 48), (1, 64), (2, 32), (2, 64)])
@@ -185,12 +226,14 @@ def test_masked_small_all_rows(expected_m):
     assert H.untouched(d)[~valid].all(), "rows at or beyond masked_m were written"
 
 
-@pytest.mark.parametrize("mw,bn", [(1, 64), (1, 224), (2, 64), (2, 128)])
-def test_masked_forced_shapes(mw, bn):
-    prob = inputs.make_masked(3, 300, 256, 256, seed=32 + bn, masked_m=[300, 0, 129])
+@pytest.mark.parametrize("mw,bn,pair", [(1, 64, 0), (1, 224, 0), (2, 64, 0), (2, 128, 0),
+                                        (1, 128, 1), (1, 256, 1)])
+def test_masked_forced_shapes(mw, bn, pair):
+    prob = inputs.make_masked(4, 300, 256, 256, seed=32 + bn + pair,
+                              masked_m=[300, 0, 129, 257])
     ref = oracle.gemm_masked(prob.a, prob.sa, prob.b, prob.sb, prob.masked_m, prob.G,
                              prob.M_max, prob.N, prob.K)
-    fp8.force_config(128 * mw, bn)
+    force_shape(mw, bn, pair)
     try:
         d = H.run_masked(prob)
     finally:

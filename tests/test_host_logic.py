@@ -90,20 +90,27 @@ def test_block_n_example_tile_counts(lib):
             fp8.force_config(bm, bn)
             cfg = fp8.select_config(fp8.KIND_DENSE, M, N, 2048, num_sms=sms)
             assert (cfg["block_m"], cfg["block_n"], cfg["num_tiles"]) == (bm, bn, tiles)
+        # with the tile width free (one CTA per tile) on the same 132-SM
+        # part, the selector fills more SMs than 112
+        fp8.force_config(0, 0, 0, 1)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=132)
+        assert cfg["num_tiles"] <= 132 and cfg["num_tiles"] >= 128
     finally:
         fp8.force_config(0, 0)
-    # unforced on the same 132-SM part, the selector fills more SMs than 112
-    cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=132)
-    assert cfg["num_tiles"] <= 132 and cfg["num_tiles"] >= 128
 
 
 def test_selector_fills_b200_for_prefill_shapes(lib):
-    cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=148)
-    assert cfg["num_tiles"] <= 148 and cfg["num_tiles"] >= 128
-    assert cfg["block_n"] % 16 == 0 and cfg["block_n"] & (cfg["block_n"] - 1) != 0
+    try:
+        fp8.force_config(0, 0, 0, 1)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=148)
+        assert cfg["num_tiles"] <= 148 and cfg["num_tiles"] >= 128
+        assert cfg["block_n"] % 16 == 0 and cfg["block_n"] & (cfg["block_n"] - 1) != 0
+    finally:
+        fp8.force_config(0, 0)
     cfg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
-    waves = -(-cfg["num_tiles"] // 148)
-    assert cfg["num_tiles"] / (waves * 148) > 0.95
+    ctas = cfg["num_tiles"] * cfg["cta_pair"]
+    waves = -(-ctas // 148)
+    assert ctas / (waves * 148) > 0.95
 
 
 def test_selector_invariants_and_determinism(lib):
@@ -118,14 +125,21 @@ def test_selector_invariants_and_determinism(lib):
         b = fp8.select_config(kind, M, N, K, G, em, 148)
         assert a == b
         assert a["block_m"] in (128, 256) and a["block_n"] % 16 == 0
-        assert 16 <= a["block_n"] <= 256 and (a["block_m"] == 128 or a["block_n"] <= 128)
+        assert a["cta_pair"] in (1, 2)
+        pair = a["cta_pair"] == 2
+        assert 16 <= a["block_n"] <= 256 and (a["block_m"] == 128 or a["block_n"] <= 128 or pair)
         assert a["stages"] >= 2
         assert a["smem_bytes"] <= 232448
-        assert a["tmem_cols"] >= 2 * (a["block_m"] // 128) * a["block_n"]
+        # TMEM per CTA: at least two K-block partials of the CTA's 128 or 256 rows
+        rows_per_cta = 128 if pair else a["block_m"]
+        assert a["tmem_cols"] >= 2 * (rows_per_cta // 128) * a["block_n"]
         assert a["tmem_cols"] <= 512 and a["tmem_cols"] & (a["tmem_cols"] - 1) == 0
         assert 1 <= a["grid"] <= 148
+        if pair:
+            assert a["block_m"] == 256 and a["split"] == 1 and a["grid"] % 2 == 0
+            assert a["block_n"] % 32 == 0
         if kind == fp8.KIND_CONTIGUOUS:
-            assert a["block_m"] == 128
+            assert a["block_m"] == 128 and not pair
 
 
 def test_decode_shape_uses_split_k_in_one_wave(lib):
@@ -153,8 +167,38 @@ def test_force_config_rejects_unbuilt_shapes(lib):
     with pytest.raises(fp8.Fp8NtError):
         fp8.force_config(128, 120)
     with pytest.raises(fp8.Fp8NtError):
-        fp8.force_config(256, 256)
+        fp8.force_config(256, 256, 0, 1)  # one CTA cannot hold 256 x 256 in TMEM
+    with pytest.raises(fp8.Fp8NtError):
+        fp8.force_config(256, 112, 0, 2)  # no pair kernel of that width
+    with pytest.raises(fp8.Fp8NtError):
+        fp8.force_config(0, 0, 0, 3)
     fp8.force_config(0, 0)
+
+
+def test_cta_pair_selection(lib):
+    # automatic selection keeps one CTA per tile
+    assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["cta_pair"] == 1
+    try:
+        fp8.force_config(256, 256, 0, 2)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
+        assert (cfg["block_m"], cfg["block_n"], cfg["cta_pair"]) == (256, 256, 2)
+        assert cfg["num_tiles"] == 16 * 28 and cfg["grid"] == 148
+        # B is split between the pair: 16 KB of A + 16 KB of B per stage
+        fp8.force_config(256, 128, 0, 2)
+        cfg2 = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
+        assert cfg2["cta_pair"] == 2 and cfg2["stages"] > cfg["stages"]
+        fp8.force_config(256, 128, 0, 1)
+        assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["cta_pair"] == 1
+        # tiles fewer than pairs: one pair per tile
+        fp8.force_config(256, 256, 0, 2)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 300, 1024, 512, num_sms=148)
+        assert cfg["num_tiles"] == 2 * 4 and cfg["grid"] == 16
+        # a pair never serves the contiguous layout (tiles could straddle experts)
+        fp8.force_config(0, 0, 0, 2)
+        with pytest.raises(fp8.Fp8NtError):
+            fp8.select_config(fp8.KIND_CONTIGUOUS, 128 * 40, 4096, 7168, 8, num_sms=148)
+    finally:
+        fp8.force_config(0, 0)
 
 
 def test_num_sms_bound(lib):
