@@ -36,6 +36,7 @@ constexpr int kNumCandidates = sizeof(kCandidates) / sizeof(kCandidates[0]);
 constexpr int kDefaultSms = 148;           // B200
 constexpr int kDefaultMaxSmem = 232448;    // 227 KB opt-in per block on sm_100
 constexpr int kMaxStages = 12;
+static_assert(kMaxStages <= DONE_RING, "the done ring must cover every operand stage");
 constexpr int kMinStages = 2;
 constexpr int kMaxSplit = 4;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull; // 2 s per pipeline wait

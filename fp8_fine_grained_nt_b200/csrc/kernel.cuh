@@ -309,10 +309,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const SmemPlan &plan = p.plan;
     const int stages = p.stages;
 
+    // full[s]: stage s holds its operands (two arrivals: the A and the B
+    // producer warp, each with its bytes); done[j]: the MMAs of K block j
+    // (counted per CTA, j mod DONE_RING) have completed, which both frees
+    // their operand stage and makes their TMEM partial readable;
+    // tmem_empty[b]: the epilogue has read TMEM buffer b.
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + plan.off_bars);
-    uint64_t *empty = full + stages;
-    uint64_t *tmem_full = empty + stages;
-    uint64_t *tmem_empty = tmem_full + MAX_TMEM_BUFS;
+    uint64_t *done = full + stages;
+    uint64_t *tmem_empty = done + DONE_RING;
     uint64_t *sb_full = tmem_empty + MAX_TMEM_BUFS;
     uint64_t *sb_empty = sb_full + 2;
     uint64_t *mma_done = sb_empty + 2;
@@ -324,12 +328,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     // ---------------------------------------------------------------- set-up
     if (threadIdx.x == 0) {
-        for (int s = 0; s < stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
+        for (int s = 0; s < stages; ++s)
+            mbar_init(&full[s], 2);
+        for (int j = 0; j < DONE_RING; ++j)
+            mbar_init(&done[j], 1);
         for (int b = 0; b < T::NBUF; ++b) {
-            mbar_init(&tmem_full[b], 1);
             // a pair's leader also counts the peer's epilogue warps
             mbar_init(&tmem_empty[b], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
         }
@@ -406,44 +409,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int kb_lo = split_k ? min(p.nkb, split_rank * p.kb_chunk) : 0;
     const int kb_hi = split_k ? min(p.nkb, kb_lo + p.kb_chunk) : p.nkb;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------ producers
+        // Warp 0 loads the A tile (and the tile's RHS scales), warp 2 the B
+        // tile: two threads issue each stage's copies, so that the issue
+        // latencies of the two overlap.
         regs_dec<REGS_PRODUCER>();
-        uint32_t stage_it = 0, tile_it = 0;
+        const bool a_side = warp == 0;
+        uint32_t it = 0, s = 0, tile_it = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
             const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
             if (!ti.valid)
                 continue;
-            // RHS scales of the whole tile: <= 3 rows of K/128 floats
-            const int slot = tile_it & 1;
-            if (!wait_bar_warp(&sb_empty[slot], ((tile_it >> 1) & 1) ^ 1, abort_flag, p))
-                break;
-            float *dst = sb_tile + slot * MAX_SB_BLOCKS * pitch;
-            for (int idx = lane; idx < MAX_SB_BLOCKS * p.nkb; idx += 32) {
-                const int j = idx / p.nkb;
-                const int kb = idx - j * p.nkb;
-                if (j < ti.sb_rows)
-                    cp_async_4(dst + j * pitch + kb, p.sb + (size_t)(ti.sb_row0 + j) * p.nkb + kb);
+            if (a_side) {
+                // RHS scales of the whole tile: <= 3 rows of K/128 floats
+                const int slot = tile_it & 1;
+                if (!wait_bar_warp(&sb_empty[slot], ((tile_it >> 1) & 1) ^ 1, abort_flag, p))
+                    break;
+                float *dst = sb_tile + slot * MAX_SB_BLOCKS * pitch;
+                for (int idx = lane; idx < MAX_SB_BLOCKS * p.nkb; idx += 32) {
+                    const int j = idx / p.nkb;
+                    const int kb = idx - j * p.nkb;
+                    if (j < ti.sb_rows)
+                        cp_async_4(dst + j * pitch + kb, p.sb + (size_t)(ti.sb_row0 + j) * p.nkb + kb);
+                }
+                cp_async_mbar_arrive_noinc(&sb_full[slot]);
+                ++tile_it;
             }
-            cp_async_mbar_arrive_noinc(&sb_full[slot]);
-
-            // A / B per K block.  Lane 0 copies B, lanes 1..halves the A
-            // halves: one instruction issues all of a stage's copies.
+            // A: lanes 0..halves-1 copy the 128-row halves; B: lane 0
             const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
-            const uint32_t ab_bytes = halves * T::A_HALF_BYTES + T::B_BYTES;
-            const bool copier = lane <= halves;
-            const CUtensorMap *my_map = lane == 0 ? &tmap_b : &tmap_a;
-            const int my_row = lane == 0 ? ti.b_row0 : ti.a_row0 + (lane - 1) * HALF_M;
-            const uint32_t my_off = lane == 0 ? plan.a_bytes : (uint32_t)(lane - 1) * T::A_HALF_BYTES;
+            const uint32_t bytes = a_side ? halves * T::A_HALF_BYTES : T::B_BYTES;
+            const bool copier = a_side ? lane < halves : lane == 0;
+            const CUtensorMap *my_map = a_side ? &tmap_a : &tmap_b;
+            const int my_row = a_side ? ti.a_row0 + lane * HALF_M : ti.b_row0;
+            const uint32_t my_off = a_side ? (uint32_t)lane * T::A_HALF_BYTES : plan.a_bytes;
             for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                const int s = (int)(stage_it % (uint32_t)stages);
                 int got = 1;
                 if (lane == 0) {
-                    got = wait_bar(&empty[s], ((stage_it / stages) & 1) ^ 1, abort_flag, p) ? 1 : 0;
+                    // stage s was last used by K block it - stages
+                    if (it >= (uint32_t)stages) {
+                        const uint32_t j = it - (uint32_t)stages;
+                        got = wait_bar(&done[j % DONE_RING], (j / DONE_RING) & 1, abort_flag, p) ? 1 : 0;
+                    }
                     // a pair's leader expects both CTAs' bytes on its barrier
                     if (got && leader)
-                        mbar_arrive_expect_tx(&full[s], PAIR ? 2 * ab_bytes : ab_bytes);
+                        mbar_arrive_expect_tx(&full[s], PAIR ? 2 * bytes : bytes);
                 }
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (!got) {
@@ -451,22 +462,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 if (copier) {
-                    uint8_t *dst = smem + plan.off_stages + (uint32_t)s * plan.stage_bytes + my_off;
+                    uint8_t *dst = smem + plan.off_stages + s * plan.stage_bytes + my_off;
                     if constexpr (PAIR)
                         tma_load_2d_pair(dst, my_map, map_shared_rank(smem_addr(&full[s]), 0u),
                                          kb * BLOCK_K, my_row);
                     else
                         tma_load_2d(dst, my_map, &full[s], kb * BLOCK_K, my_row);
                 }
-                ++stage_it;
+                ++it;
+                if (++s == (uint32_t)stages)
+                    s = 0;
             }
-            ++tile_it;
         }
-        // Drain: every copy issued must land before the CTA exits.
+        // Drain: every copy issued must land before the CTA exits (the full
+        // barriers count both producers' bytes, and a peer's copies are
+        // counted on the leader's barriers).
         cp_async_wait_all();
-        if (lane == 0 && leader) { // a peer's copies are drained through the leader's barriers
-            const uint32_t n = stage_it < (uint32_t)stages ? stage_it : (uint32_t)stages;
-            for (uint32_t i = stage_it - n; i < stage_it; ++i)
+        if (a_side && lane == 0 && leader) {
+            const uint32_t n = it < (uint32_t)stages ? it : (uint32_t)stages;
+            for (uint32_t i = it - n; i < it; ++i)
                 wait_drain(&full[i % stages], (i / stages) & 1, abort_flag, p);
         }
     } else if (warp == 1) {
@@ -474,7 +488,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         regs_dec<REGS_PRODUCER>();
         if (lane == 0 && leader) { // a pair's MMAs are issued by the leader alone
             constexpr uint32_t idesc = make_idesc(BN, PAIR ? 2 * HALF_M : HALF_M);
-            uint32_t stage_it = 0, kb_it = 0;
+            // descriptors of stage 0; a stage, an M half and a K step move
+            // the start-address field (address / 16, 14 bits: no carry for
+            // shared-memory addresses)
+            const uint64_t a_desc0 = make_sdesc(smem_addr(smem + plan.off_stages));
+            const uint64_t b_desc0 = make_sdesc(smem_addr(smem + plan.off_stages) + plan.a_bytes);
+            const uint32_t stage_step = plan.stage_bytes >> 4;
+            uint32_t kb_it = 0, s = 0, phase = 0;
             bool ok = true;
             for (int t = t_first; ok && t < num_tiles; t += t_stride) {
                 const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
@@ -482,8 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     continue;
                 const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    const int s = (int)(stage_it % (uint32_t)stages);
-                    if (!wait_bar(&full[s], (stage_it / stages) & 1, abort_flag, p)) {
+                    if (!wait_bar(&full[s], phase, abort_flag, p)) {
                         ok = false;
                         break;
                     }
@@ -504,33 +523,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         }
                     }
                     tc_fence_after();
-                    const uint32_t a_base =
-                        smem_addr(smem + plan.off_stages + (uint32_t)s * plan.stage_bytes);
-                    const uint32_t b_base = a_base + plan.a_bytes;
+                    const uint64_t a_desc = a_desc0 + s * stage_step;
+                    const uint64_t b_desc = b_desc0 + s * stage_step;
                     for (int h = 0; h < halves; ++h) {
                         const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS + h * BN);
 #pragma unroll
                         for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
-                            const uint64_t ad = make_sdesc(a_base + h * T::A_HALF_BYTES + k * MMA_K);
-                            const uint64_t bd = make_sdesc(b_base + k * MMA_K);
+                            const uint64_t ad = a_desc + (uint64_t)((h * T::A_HALF_BYTES + k * MMA_K) >> 4);
+                            const uint64_t bd = b_desc + (uint64_t)((k * MMA_K) >> 4);
                             if constexpr (PAIR)
                                 mma_f8f6f4_pair(d, ad, bd, idesc, k > 0 ? 1u : 0u);
                             else
                                 mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
                         }
                     }
-                    // every buffer completes one phase per use (the epilogue
-                    // waits only for a group's last one); a pair's commits
-                    // reach both CTAs
-                    if constexpr (PAIR) {
-                        mma_commit_pair_mc(&empty[s], 0x3);
-                        mma_commit_pair_mc(&tmem_full[buf], 0x3);
-                    } else {
-                        mma_commit(&empty[s]);
-                        mma_commit(&tmem_full[buf]);
-                    }
-                    ++stage_it;
+                    // one commit per K block frees its stage and publishes its
+                    // partial (a pair's commit reaches both CTAs)
+                    if constexpr (PAIR)
+                        mma_commit_pair_mc(&done[kb_it % DONE_RING], 0x3);
+                    else
+                        mma_commit(&done[kb_it % DONE_RING]);
                     ++kb_it;
+                    if (++s == (uint32_t)stages) {
+                        s = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
             // Drain: all MMAs complete before TMEM is released.
@@ -541,7 +558,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             wait_drain(mma_done, 0, abort_flag, p);
         }
     } else if (warp < FIRST_EPI_WARP) {
-        regs_dec<REGS_PRODUCER>(); // warps 2-3: idle until the end
+        regs_dec<REGS_PRODUCER>(); // warp 3: idle until the end
     } else {
         // ------------------------------------------------------------ epilogue
         regs_inc<REGS_EPILOGUE>();
@@ -601,7 +618,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             };
             // wait for K block `it`'s partial in TMEM
             auto wait_full = [&](uint32_t it) {
-                const bool r = wait_bar_warp(&tmem_full[it % T::NBUF], (it / T::NBUF) & 1, abort_flag, p);
+                const bool r = wait_bar_warp(&done[it % DONE_RING], (it / DONE_RING) & 1, abort_flag, p);
                 tc_fence_after();
                 return r;
             };

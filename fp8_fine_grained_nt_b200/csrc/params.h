@@ -17,11 +17,13 @@ constexpr int NUM_EPI_WARPS = 8;
 constexpr int MAX_SB_BLOCKS = 3;      // a BLOCK_N <= 256 tile spans at most 3 sb blocks
 constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int MAX_TMEM_BUFS = 16;      // K-block partial buffers in TMEM (ring)
+constexpr int DONE_RING = 16;          // "K block done" barriers; >= stages and >= TMEM buffers
+static_assert(DONE_RING >= MAX_TMEM_BUFS, "the done ring must cover every TMEM buffer");
 constexpr uint32_t OUT_STAGE_BYTES = 2048; // 32 rows x 32 BF16 columns per epilogue warp
 constexpr int RED_PAD = 4;             // FP32 padding per row of the split-K partial tile
 constexpr int MAX_SPLIT = 8;           // split-K CTAs per cluster (portable cluster size)
-constexpr int REGS_PRODUCER = 56;     // per-thread registers after setmaxnreg
-constexpr int REGS_EPILOGUE = 224;
+constexpr int REGS_PRODUCER = 40;     // per-thread registers after setmaxnreg
+constexpr int REGS_EPILOGUE = 232;
 constexpr int REGS_AT_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
 
 static_assert(4 * 32 * REGS_PRODUCER + 8 * 32 * REGS_EPILOGUE <= NUM_THREADS * REGS_AT_LAUNCH,
@@ -96,9 +98,9 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     p.off_prefix = align_up_u32(off, 16);
     off = p.off_prefix + 4u * (uint32_t)prefix_ints;
     p.off_bars = align_up_u32(off, 8);
-    // full/empty per stage, TMEM full/empty per partial buffer, sb
-    // full/empty x2, one "all MMAs done" barrier
-    off = p.off_bars + 8u * (2u * stages + 2u * MAX_TMEM_BUFS + 4u + 1u);
+    // full per stage, the ring of "K block done" barriers, TMEM empty per
+    // partial buffer, sb full/empty x2, one "all MMAs done" barrier
+    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 4u + 1u);
     p.off_misc = align_up_u32(off, 16);
     p.total = p.off_misc + 16;
     return p;
