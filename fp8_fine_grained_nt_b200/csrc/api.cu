@@ -154,16 +154,46 @@ struct Problem {
     int expected_m; // masked only
 };
 
-// Rough cycle estimate of a (MW, BN, split, pair) choice on `sms` SMs: whole
-// waves of CTAs, each working through its K blocks, a K block limited by the
-// tensor pipe (one kind::f8f6f4 MMA issues every max(64, BN/2) cycles, four
-// per 128-row block at K=32), operand delivery (~64 B/clk/SM from L2; a CTA
-// of a pair loads half of B) or the promotion FMAs (BN cycles per 128 rows),
-// plus a fixed per-block pipeline latency; split-K adds the cluster
-// reduction.
+// Relative cost of one K block of a tile, by tile shape, measured on B200
+// (dense 4096x7168x2048, 256x7168x2048, masked and contiguous shapes; time
+// per K block per wave, BLOCK_N = 256 with one 128-row CTA = 1.0).  It is
+// nearly flat in BLOCK_N: a K block is bound by the per-K-block pipeline
+// (operand ring latency, TMEM partial reads, promotion), not by MMA rate or
+// L2 bandwidth, so wide tiles and few waves win.  Two 128-row halves in one
+// CTA cost more per K block; narrow tiles (<= 64 columns per K block) less.
+double kb_cost_factor(int mw, int bn, int halves)
+{
+    if (mw == 2 && halves == 2) {
+        switch (bn) {
+        case 64: return 1.05;
+        case 96: return 1.18;
+        case 112: return 1.26;
+        case 128: return 1.18;
+        default: return 1.2;
+        }
+    }
+    switch (bn) {
+    case 64: return 0.70;
+    case 96: return 0.97;
+    case 112: return 0.99;
+    case 128: return 0.99;
+    case 160: return 0.94;
+    case 192: return 1.02;
+    case 224: return 1.08;
+    case 256: return 1.0;
+    default: return bn < 64 ? 0.6 : 1.0;
+    }
+}
+
+// Cycle estimate of a (MW, BN, split, pair) choice on `sms` SMs: whole
+// waves of CTAs (a CTA pair takes two SMs), each working through its K
+// blocks at ~1300 cycles x kb_cost_factor per K block, plus a per-tile cost
+// (pipeline ramp, and the BF16 store, which grows with the tile's size);
+// split-K adds the cluster reduction.
 double estimate_cycles(const Problem &pb, int mw, int bn, int split, int pair, int stages, int sms,
                        int *tiles_out)
 {
+    (void)stages;
     const int bm = pair ? 256 : 128 * mw;
     const int nkb = pb.K / 128;
     long m_blocks;
@@ -183,16 +213,10 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int split, int pair, i
     const long ctas = tiles * split * (pair ? 2 : 1);
     const long waves = (ctas + sms - 1) / sms;
     const int halves = (mw == 2 && rows_eff > 128) ? 2 : 1;
-    const double mma = 4.0 * halves * (bn / 2 > 64 ? bn / 2 : 64);
-    const int a_rows = pair ? 128 : rows_eff;
-    const double l2 = (double)(a_rows + (pair ? bn / 2 : bn)) * 128.0 / 64.0;
-    const double epi = (double)bn * halves;
-    (void)stages;
-    double per_kb = mma > l2 ? mma : l2;
-    per_kb = per_kb > epi ? per_kb : epi;
-    per_kb += 250.0;
     const int kb_per_cta = ceil_div(nkb, split);
-    double tile = kb_per_cta * per_kb + 1500.0;
+    const int cta_rows = pair ? 128 : (rows_eff < 128 * mw ? rows_eff : 128 * mw);
+    double tile = kb_per_cta * 1300.0 * kb_cost_factor(pair ? 1 : mw, bn, halves) + 1500.0 +
+                  3500.0 * bn * cta_rows / (256.0 * 128.0);
     if (split > 1)
         tile += 800.0 + (double)bm * bn * 4.0 * split / 256.0 / split;
     if (tiles_out)
@@ -365,7 +389,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     const int groups = pb.kind == DG_KIND_DENSE ? 1 : pb.groups;
     const int ld_sa = get_tma_aligned_size(pb.M, 4);
 
-    CUtensorMap tmap_a, tmap_b;
+    CUtensorMap tmap_a, tmap_b, tmap_sa;
     const long a_rows = pb.kind == DG_KIND_MASKED ? (long)groups * pb.M : pb.M;
     const long b_rows = (long)groups * pb.N;
     if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, a_rows, pb.K, 128,
@@ -375,6 +399,16 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     const uint32_t b_box_rows = cand->pair ? cfg.block_n / 2 : cfg.block_n;
     if ((st = make_tmap_2d(&tmap_b, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, b_rows, pb.K, 128,
                            b_box_rows, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+        return st;
+    // LHS scales as a [sa_groups * K/128][ld_sa] FP32 matrix (only the
+    // masked form has one scale block per group; the contiguous form's rows
+    // are already concatenated); one box holds a CTA's rows for
+    // SA_SLOT_BYTES / (rows * 4) consecutive K blocks
+    const long sa_groups = pb.kind == DG_KIND_MASKED ? groups : 1;
+    const uint32_t sa_box_rows = cand->pair ? 128u : (uint32_t)cfg.block_m;
+    if ((st = make_tmap_2d(&tmap_sa, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)ld_sa,
+                           (uint64_t)sa_groups * nkb, (uint64_t)ld_sa, sa_box_rows,
+                           SA_SLOT_BYTES / (sa_box_rows * 4u), CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
         return st;
 
     Params p;
@@ -405,6 +439,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     LaunchArgs args;
     args.tmap_a = &tmap_a;
     args.tmap_b = &tmap_b;
+    args.tmap_sa = &tmap_sa;
     args.params = &p;
     args.grid = cfg.grid;
     args.cluster = cand->pair ? 2 : cfg.split;

@@ -44,6 +44,10 @@ struct KernelTraits {
     // rows of the tile a CTA (or, with PAIR, a CTA pair) computes
     static constexpr int BLOCK_M = PAIR ? 2 * HALF_M : MW * HALF_M;
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN; // rows of B each CTA loads
+    // LHS scales reach shared memory in blocks of SA_GROUP K blocks x
+    // SA_ROWS rows (the CTA's rows), SA_SLOT_BYTES per ring slot
+    static constexpr int SA_ROWS = PAIR ? HALF_M : MW * HALF_M;
+    static constexpr int SA_GROUP = (int)SA_SLOT_BYTES / (SA_ROWS * 4);
     static constexpr int BUF_COLS = MW * BN;                 // TMEM columns per K-block buffer
     // ring of K-block partial buffers in TMEM: as many as fit, at most 16
     static constexpr int NBUF = (512 / BUF_COLS) < MAX_TMEM_BUFS ? (512 / BUF_COLS) : MAX_TMEM_BUFS;
@@ -297,7 +301,8 @@ __device__ __forceinline__ void fma_range_any(float (&acc)[NC], const float (&v)
 template <int MW, int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ Params p)
+                    const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ Params p)
 {
     using T = KernelTraits<MW, BN, PAIR>;
     extern __shared__ uint8_t smem_raw[];
@@ -319,11 +324,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t *tmem_empty = done + DONE_RING;
     uint64_t *sb_full = tmem_empty + MAX_TMEM_BUFS;
     uint64_t *sb_empty = sb_full + 2;
-    uint64_t *mma_done = sb_empty + 2;
+    uint64_t *sa_full = sb_empty + 2;  // LHS-scale ring (2 slots)
+    uint64_t *sa_empty = sa_full + 2;
+    uint64_t *mma_done = sa_empty + 2;
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + plan.off_misc);
     volatile uint32_t *abort_flag = misc + 1;
     int *prefix = reinterpret_cast<int *>(smem + plan.off_prefix);
     float *sb_tile = reinterpret_cast<float *>(smem + plan.off_sb);
+    float *sa_ring = reinterpret_cast<float *>(smem + plan.off_sa);
     const int pitch = (int)plan.sb_pitch;
 
     // ---------------------------------------------------------------- set-up
@@ -339,6 +347,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sb_full[b], 32);
             mbar_init(&sb_empty[b], NUM_EPI_WARPS);
+            mbar_init(&sa_full[b], 1);
+            mbar_init(&sa_empty[b], NUM_EPI_WARPS);
         }
         mbar_init(mma_done, 1);
         misc[1] = 0u;
@@ -347,6 +357,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
+        tma_prefetch_desc(&tmap_sa);
     }
     if (warp == 1) {
         if constexpr (PAIR) {
@@ -411,32 +422,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0 || warp == 2) {
         // ------------------------------------------------------------ producers
-        // Warp 0 loads the A tile (and the tile's RHS scales), warp 2 the B
-        // tile: two threads issue each stage's copies, so that the issue
-        // latencies of the two overlap.
+        // Warp 0 loads the A tile, warp 2 the B tile: two threads issue each
+        // stage's copies, so that the issue latencies of the two overlap.
         regs_dec<REGS_PRODUCER>();
         const bool a_side = warp == 0;
-        uint32_t it = 0, s = 0, tile_it = 0;
+        uint32_t it = 0, s = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
             const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
             if (!ti.valid)
                 continue;
-            if (a_side) {
-                // RHS scales of the whole tile: <= 3 rows of K/128 floats
-                const int slot = tile_it & 1;
-                if (!wait_bar_warp(&sb_empty[slot], ((tile_it >> 1) & 1) ^ 1, abort_flag, p))
-                    break;
-                float *dst = sb_tile + slot * MAX_SB_BLOCKS * pitch;
-                for (int idx = lane; idx < MAX_SB_BLOCKS * p.nkb; idx += 32) {
-                    const int j = idx / p.nkb;
-                    const int kb = idx - j * p.nkb;
-                    if (j < ti.sb_rows)
-                        cp_async_4(dst + j * pitch + kb, p.sb + (size_t)(ti.sb_row0 + j) * p.nkb + kb);
-                }
-                cp_async_mbar_arrive_noinc(&sb_full[slot]);
-                ++tile_it;
-            }
             // A: lanes 0..halves-1 copy the 128-row halves; B: lane 0
             const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
             const uint32_t bytes = a_side ? halves * T::A_HALF_BYTES : T::B_BYTES;
@@ -477,7 +472,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Drain: every copy issued must land before the CTA exits (the full
         // barriers count both producers' bytes, and a peer's copies are
         // counted on the leader's barriers).
-        cp_async_wait_all();
         if (a_side && lane == 0 && leader) {
             const uint32_t n = it < (uint32_t)stages ? it : (uint32_t)stages;
             for (uint32_t i = it - n; i < it; ++i)
@@ -557,8 +551,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 mma_commit(mma_done);
             wait_drain(mma_done, 0, abort_flag, p);
         }
-    } else if (warp < FIRST_EPI_WARP) {
-        regs_dec<REGS_PRODUCER>(); // warp 3: idle until the end
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ scales
+        // Per tile, the RHS scales (<= 3 rows of K/128 floats, cp.async by
+        // all lanes); per SA_GROUP K blocks, the LHS scales of the CTA's
+        // rows (one TMA box of SA_GROUP x SA_ROWS floats, lane 0) into a
+        // two-slot ring that the epilogue releases.
+        regs_dec<REGS_PRODUCER>();
+        uint32_t tile_it = 0, grp_it = 0;
+        bool ok = true;
+        for (int t = t_first; ok && t < num_tiles; t += t_stride) {
+            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+            if (!ti.valid)
+                continue;
+            const int slot = tile_it & 1;
+            if (!wait_bar_warp(&sb_empty[slot], ((tile_it >> 1) & 1) ^ 1, abort_flag, p))
+                break;
+            float *dst = sb_tile + slot * MAX_SB_BLOCKS * pitch;
+            for (int idx = lane; idx < MAX_SB_BLOCKS * p.nkb; idx += 32) {
+                const int j = idx / p.nkb;
+                const int kb = idx - j * p.nkb;
+                if (j < ti.sb_rows)
+                    cp_async_4(dst + j * pitch + kb, p.sb + (size_t)(ti.sb_row0 + j) * p.nkb + kb);
+            }
+            cp_async_mbar_arrive_noinc(&sb_full[slot]);
+            ++tile_it;
+            for (int k0 = kb_lo; k0 < kb_hi; k0 += T::SA_GROUP) {
+                const uint32_t gs = grp_it & 1;
+                int got = 1;
+                if (lane == 0) {
+                    got = wait_bar(&sa_empty[gs], ((grp_it >> 1) & 1) ^ 1, abort_flag, p) ? 1 : 0;
+                    if (got) {
+                        mbar_arrive_expect_tx(&sa_full[gs], SA_SLOT_BYTES);
+                        tma_load_2d(sa_ring + gs * (SA_SLOT_BYTES / 4), &tmap_sa, &sa_full[gs], ti.m0,
+                                    ti.sa_y0 + k0);
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                ++grp_it;
+            }
+        }
+        // Drain: the last copies must land before the CTA exits.
+        cp_async_wait_all();
+        if (lane == 0) {
+            const uint32_t n = grp_it < 2u ? grp_it : 2u;
+            for (uint32_t i = grp_it - n; i < grp_it; ++i)
+                wait_drain(&sa_full[i & 1], (i >> 1) & 1, abort_flag, p);
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         regs_inc<REGS_EPILOGUE>();
@@ -570,7 +612,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int half = (MW == 1) ? 0 : wg;
         const int row_in_tile = half * HALF_M + q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        uint32_t kb_it = 0, tile_it = 0;
+        uint32_t kb_it = 0, tile_it = 0, sa_it = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
             const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
@@ -588,23 +630,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int lo = (cbase >> 7) - (ti.n0 >> 7);
             const int t_split = ((cbase >> 7) + 1) * 128 - cbase;
             const bool split = t_split < NC;
-            // LHS scales of this thread's row, read from global memory four
-            // K blocks ahead of use (rows past the scale tensor's leading
-            // dimension read nothing; they are never stored)
-            const int sa_row = ti.m0 + row_in_tile;
-            const float *sa_ptr = p.sa + (size_t)ti.sa_y0 * p.ld_sa + sa_row;
-            const bool sa_ok = sa_row < p.ld_sa;
-            auto sa_load = [&](int kb) {
-                return (sa_ok && kb < kb_hi) ? __ldg(sa_ptr + (size_t)kb * p.ld_sa) : 0.0f;
-            };
-            float sa_q0 = sa_load(kb_lo), sa_q1 = sa_load(kb_lo + 1), sa_q2 = sa_load(kb_lo + 2),
-                  sa_q3 = sa_load(kb_lo + 3);
+            // LHS scales of this thread's row come from the shared-memory
+            // ring, SA_GROUP K blocks per slot; K blocks are consumed in
+            // order, so a slot is awaited at its first K block and released
+            // after its last (rows past M read the zero fill and are never
+            // stored)
             auto scales = [&](int kb, float &s_lo, float &s_hi) {
-                const float sa_v = sa_q0;
-                sa_q0 = sa_q1;
-                sa_q1 = sa_q2;
-                sa_q2 = sa_q3;
-                sa_q3 = sa_load(kb + 4);
+                const int gpos = (kb - kb_lo) % T::SA_GROUP;
+                const uint32_t gs = sa_it & 1;
+                if (gpos == 0)
+                    wait_bar_warp(&sa_full[gs], (sa_it >> 1) & 1, abort_flag, p);
+                const float sa_v = sa_ring[gs * (SA_SLOT_BYTES / 4) + gpos * T::SA_ROWS + row_in_tile];
+                if (gpos == T::SA_GROUP - 1 || kb == kb_hi - 1) {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&sa_empty[gs]);
+                    ++sa_it;
+                }
                 s_lo = sa_v * sbt[lo * pitch + kb];
                 s_hi = sa_v * sbt[(lo + 1) * pitch + kb];
             };

@@ -20,6 +20,7 @@ constexpr int MAX_TMEM_BUFS = 16;      // K-block partial buffers in TMEM (ring)
 constexpr int DONE_RING = 16;          // "K block done" barriers; >= stages and >= TMEM buffers
 static_assert(DONE_RING >= MAX_TMEM_BUFS, "the done ring must cover every TMEM buffer");
 constexpr uint32_t OUT_STAGE_BYTES = 2048; // 32 rows x 32 BF16 columns per epilogue warp
+constexpr uint32_t SA_SLOT_BYTES = 4096;   // one slot of the LHS-scale ring (2 slots)
 constexpr int RED_PAD = 4;             // FP32 padding per row of the split-K partial tile
 constexpr int MAX_SPLIT = 8;           // split-K CTAs per cluster (portable cluster size)
 constexpr int REGS_PRODUCER = 40;     // per-thread registers after setmaxnreg
@@ -39,6 +40,7 @@ struct SmemPlan {
     uint32_t off_stages;    // 1024-aligned
     uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
     uint32_t sb_pitch;      // floats per sb row in smem (nkb rounded up to 4)
+    uint32_t off_sa;        // LHS-scale ring: 2 x SA_SLOT_BYTES
     uint32_t off_out;       // output staging: one 2 KB buffer per epilogue warp
     uint32_t off_red;       // split-K: this CTA's FP32 partial tile, rows padded by RED_PAD
     uint32_t off_prefix;    // masked: (G + 1) ints of per-group tile prefix sums
@@ -90,6 +92,8 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     p.sb_pitch = align_up_u32((uint32_t)nkb, 4);
     p.off_sb = align_up_u32(off, 128);
     off = p.off_sb + 2u * MAX_SB_BLOCKS * p.sb_pitch * 4u;
+    p.off_sa = align_up_u32(off, 128);
+    off = p.off_sa + 2u * SA_SLOT_BYTES;
     p.off_out = align_up_u32(off, 1024);
     off = p.off_out + NUM_EPI_WARPS * OUT_STAGE_BYTES;
     p.off_red = align_up_u32(off, 128);
@@ -99,8 +103,8 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     off = p.off_prefix + 4u * (uint32_t)prefix_ints;
     p.off_bars = align_up_u32(off, 8);
     // full per stage, the ring of "K block done" barriers, TMEM empty per
-    // partial buffer, sb full/empty x2, one "all MMAs done" barrier
-    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 4u + 1u);
+    // partial buffer, sb and sa full/empty x2, one "all MMAs done" barrier
+    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u);
     p.off_misc = align_up_u32(off, 16);
     p.total = p.off_misc + 16;
     return p;
