@@ -389,7 +389,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     const int groups = pb.kind == DG_KIND_DENSE ? 1 : pb.groups;
     const int ld_sa = get_tma_aligned_size(pb.M, 4);
 
-    CUtensorMap tmap_a, tmap_b, tmap_sa;
+    CUtensorMap tmap_a, tmap_b, tmap_sa, tmap_d;
     const long a_rows = pb.kind == DG_KIND_MASKED ? (long)groups * pb.M : pb.M;
     const long b_rows = (long)groups * pb.N;
     if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, a_rows, pb.K, 128,
@@ -409,6 +409,12 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     if ((st = make_tmap_2d(&tmap_sa, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)ld_sa,
                            (uint64_t)sa_groups * nkb, (uint64_t)ld_sa, sa_box_rows,
                            SA_SLOT_BYTES / (sa_box_rows * 4u), CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
+        return st;
+    // D as a [rows][N] BF16 matrix; the epilogue stores 32 x 32 boxes staged
+    // with the 64-byte swizzle (elements past the tensor are not written)
+    const long d_rows = pb.kind == DG_KIND_MASKED ? (long)groups * pb.M : pb.M;
+    if ((st = make_tmap_2d(&tmap_d, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pb.N, d_rows, pb.N, 32,
+                           32, CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
         return st;
 
     Params p;
@@ -440,6 +446,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     args.tmap_a = &tmap_a;
     args.tmap_b = &tmap_b;
     args.tmap_sa = &tmap_sa;
+    args.tmap_d = &tmap_d;
     args.params = &p;
     args.grid = cfg.grid;
     args.cluster = cand->pair ? 2 : cfg.split;

@@ -73,7 +73,8 @@ cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN, FP8NT_PAIR)(const LaunchArgs &args)
         attr[0].val.clusterDim.z = 1;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, kernel, *args.tmap_a, *args.tmap_b, *args.tmap_sa, *args.params);
+    return cudaLaunchKernelEx(&cfg, kernel, *args.tmap_a, *args.tmap_b, *args.tmap_sa, *args.tmap_d,
+                              *args.params);
 }
 
 } // namespace fp8nt

@@ -48,6 +48,8 @@ struct KernelTraits {
     // SA_ROWS rows (the CTA's rows), SA_SLOT_BYTES per ring slot
     static constexpr int SA_ROWS = PAIR ? HALF_M : MW * HALF_M;
     static constexpr int SA_GROUP = (int)SA_SLOT_BYTES / (SA_ROWS * 4);
+    // 32-column chunks of an epilogue thread's columns (output staging)
+    static constexpr int OUT_CHUNKS = ((MW == 1 ? BN / 2 : BN) + 31) / 32;
     static constexpr int BUF_COLS = MW * BN;                 // TMEM columns per K-block buffer
     // ring of K-block partial buffers in TMEM: as many as fit, at most 16
     static constexpr int NBUF = (512 / BUF_COLS) < MAX_TMEM_BUFS ? (512 / BUF_COLS) : MAX_TMEM_BUFS;
@@ -302,7 +304,8 @@ template <int MW, int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
-                    const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ Params p)
+                    const __grid_constant__ CUtensorMap tmap_sa,
+                    const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ Params p)
 {
     using T = KernelTraits<MW, BN, PAIR>;
     extern __shared__ uint8_t smem_raw[];
@@ -358,6 +361,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
         tma_prefetch_desc(&tmap_sa);
+        tma_prefetch_desc(&tmap_d);
     }
     if (warp == 1) {
         if constexpr (PAIR) {
@@ -795,17 +799,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         atomicOr(p.status, DEVERR_BAD_INDEX);
                 }
             }
-            // Each warp owns 32 rows; it passes them 32 columns at a time
-            // through a 2 KB shared buffer (16-byte pieces XOR-swizzled to
-            // avoid bank conflicts) so that the global writes are 64-byte
-            // row segments: 4 lanes per row, 8 rows per instruction.
+            // Each warp owns 32 rows and NC columns.  It writes them as BF16
+            // into its part of the tile's staging buffer, 32 columns (2 KB)
+            // per chunk: 64-byte rows whose 16-byte pieces are XOR-swizzled
+            // by (row / 2) % 4, the TMA 64-byte swizzle, which also spreads
+            // the writes over all banks.  Full chunks go out as TMA stores
+            // (asynchronous: the warp moves on to the next tile) when every
+            // row of the warp is stored, or for the dense form, whose tensor
+            // map clips the rows past M; other chunks use plain 16-byte
+            // stores of whole 64-byte row segments.
             const uint32_t row_mask = __ballot_sync(0xffffffffu, row_ok);
-            const uint32_t stg = smem_addr(smem + plan.off_out) + (uint32_t)ew * OUT_STAGE_BYTES;
+            const bool use_tma = row_mask != 0u && (row_mask == 0xffffffffu || p.kind == KIND_DENSE);
+            const uint32_t stg_w = smem_addr(smem + plan.off_out) +
+                                   (uint32_t)ew * (uint32_t)(T::OUT_CHUNKS * OUT_STAGE_BYTES);
             const int warp_row0 = ti.d_row0 + half * HALF_M + q * 32;
             const int rd_sub = lane >> 2;  // row within an 8-row group (read side)
             const int rd_piece = lane & 3; // 16-byte piece within a 64-byte row chunk
+            // the previous tile's TMA stores must have read this warp's buffer
+            if (lane == 0)
+                bulk_wait_read_all();
+            __syncwarp();
 #pragma unroll
             for (int c = 0; c < NC; c += 32) {
+                const uint32_t stg = stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (c + 8 * j < NC)
@@ -814,22 +830,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                      pack_bf16x2(acc[c + 8 * j + 2], acc[c + 8 * j + 3]),
                                      pack_bf16x2(acc[c + 8 * j + 4], acc[c + 8 * j + 5]),
                                      pack_bf16x2(acc[c + 8 * j + 6], acc[c + 8 * j + 7]));
-                __syncwarp();
-                const int col = cbase + c + 8 * rd_piece;
-                const bool col_ok = (c + 8 * rd_piece < NC) && col < p.N;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            bool issued = false;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = i * 8 + rd_sub;
-                    if (col_ok && ((row_mask >> r) & 1u)) {
-                        const uint4 v =
-                            ld_shared_v4(stg + r * 64 + ((rd_piece ^ ((r >> 1) & 3)) << 4));
-                        st_global_v4(p.D + (size_t)(warp_row0 + r) * p.N + col, v.x, v.y, v.z,
-                                     v.w);
+            for (int c = 0; c < NC; c += 32) {
+                const uint32_t stg = stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES;
+                if (use_tma && c + 32 <= NC) {
+                    if (lane == 0)
+                        tma_store_2d(&tmap_d, stg, cbase + c, warp_row0);
+                    issued = true;
+                } else if (row_mask != 0u) {
+                    const int col = cbase + c + 8 * rd_piece;
+                    const bool col_ok = (c + 8 * rd_piece < NC) && col < p.N;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = i * 8 + rd_sub;
+                        if (col_ok && ((row_mask >> r) & 1u)) {
+                            const uint4 v =
+                                ld_shared_v4(stg + r * 64 + ((rd_piece ^ ((r >> 1) & 3)) << 4));
+                            st_global_v4(p.D + (size_t)(warp_row0 + r) * p.N + col, v.x, v.y, v.z,
+                                         v.w);
+                        }
                     }
                 }
-                __syncwarp();
             }
+            if (issued && lane == 0)
+                bulk_commit_group();
         }
+        // every TMA store has completed before the CTA exits
+        if (lane == 0)
+            bulk_wait_all();
     }
 
     __syncwarp();

@@ -13,6 +13,7 @@ struct LaunchArgs {
     const CUtensorMap *tmap_a;
     const CUtensorMap *tmap_b;
     const CUtensorMap *tmap_sa;
+    const CUtensorMap *tmap_d;
     const Params *params;
     int grid;
     int cluster; // CTAs per cluster (split-K, or 2 for a CTA pair), 1 = no cluster

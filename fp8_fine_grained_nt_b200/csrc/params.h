@@ -19,7 +19,7 @@ constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int MAX_TMEM_BUFS = 16;      // K-block partial buffers in TMEM (ring)
 constexpr int DONE_RING = 16;          // "K block done" barriers; >= stages and >= TMEM buffers
 static_assert(DONE_RING >= MAX_TMEM_BUFS, "the done ring must cover every TMEM buffer");
-constexpr uint32_t OUT_STAGE_BYTES = 2048; // 32 rows x 32 BF16 columns per epilogue warp
+constexpr uint32_t OUT_STAGE_BYTES = 2048; // output staging chunk: 32 rows x 32 BF16 columns
 constexpr uint32_t SA_SLOT_BYTES = 4096;   // one slot of the LHS-scale ring (2 slots)
 constexpr int RED_PAD = 4;             // FP32 padding per row of the split-K partial tile
 constexpr int MAX_SPLIT = 8;           // split-K CTAs per cluster (portable cluster size)
@@ -41,7 +41,7 @@ struct SmemPlan {
     uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
     uint32_t sb_pitch;      // floats per sb row in smem (nkb rounded up to 4)
     uint32_t off_sa;        // LHS-scale ring: 2 x SA_SLOT_BYTES
-    uint32_t off_out;       // output staging: one 2 KB buffer per epilogue warp
+    uint32_t off_out;       // output staging: the whole BF16 tile, 2 KB chunks per epilogue warp
     uint32_t off_red;       // split-K: this CTA's FP32 partial tile, rows padded by RED_PAD
     uint32_t off_prefix;    // masked: (G + 1) ints of per-group tile prefix sums
     uint32_t off_bars;      // all mbarriers
@@ -95,7 +95,10 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     p.off_sa = align_up_u32(off, 128);
     off = p.off_sa + 2u * SA_SLOT_BYTES;
     p.off_out = align_up_u32(off, 1024);
-    off = p.off_out + NUM_EPI_WARPS * OUT_STAGE_BYTES;
+    // (split-K CTAs reduce through distributed shared memory and store
+    // directly: no output staging)
+    const uint32_t out_chunks = split_k ? 0u : (uint32_t)((mw == 1 ? bn / 2 : bn) + 31) / 32;
+    off = p.off_out + NUM_EPI_WARPS * out_chunks * OUT_STAGE_BYTES;
     p.off_red = align_up_u32(off, 128);
     if (split_k)
         off = p.off_red + (uint32_t)mw * HALF_M * (uint32_t)(bn + RED_PAD) * 4u;
