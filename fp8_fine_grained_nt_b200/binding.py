@@ -21,6 +21,7 @@ __all__ = [
     "library_path",
     "load_library",
     "gemm_fp8_fp8_bf16_nt",
+    "gemm_fp8_fp8_bf16_nt_per_tensor",
     "m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
     "m_grouped_gemm_fp8_fp8_bf16_nt_masked",
     "get_m_alignment_for_contiguous_layout",
@@ -35,6 +36,7 @@ __all__ = [
     "KIND_DENSE",
     "KIND_CONTIGUOUS",
     "KIND_MASKED",
+    "KIND_DENSE_PER_TENSOR",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +44,7 @@ _LIB_NAME = "libfp8nt.so"
 _lock = threading.Lock()
 _lib = None
 
-KIND_DENSE, KIND_CONTIGUOUS, KIND_MASKED = 0, 1, 2
+KIND_DENSE, KIND_CONTIGUOUS, KIND_MASKED, KIND_DENSE_PER_TENSOR = 0, 1, 2, 3
 
 
 class Fp8NtError(RuntimeError):
@@ -79,6 +81,7 @@ def load_library():
         lib = ctypes.CDLL(path)
         P, I = ctypes.c_void_p, ctypes.c_int
         lib.gemm_fp8_fp8_bf16_nt.argtypes = [P, P, P, P, P, I, I, I, P]
+        lib.gemm_fp8_fp8_bf16_nt_per_tensor.argtypes = [P, P, P, P, P, I, I, I, P]
         lib.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         lib.m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.get_m_alignment_for_contiguous_layout.argtypes = []
@@ -145,6 +148,28 @@ def gemm_fp8_fp8_bf16_nt(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor,
         raise ValueError("shape mismatch between a, b and d")
     _check(load_library().gemm_fp8_fp8_bf16_nt(*args, M, N, K, _stream_ptr(stream)),
            "gemm_fp8_fp8_bf16_nt")
+    return d
+
+
+def gemm_fp8_fp8_bf16_nt_per_tensor(a: torch.Tensor, scale_a: torch.Tensor, b: torch.Tensor,
+                                    scale_b: torch.Tensor, d: torch.Tensor,
+                                    stream=None) -> torch.Tensor:
+    """D[M,N] (bf16) = scale_a * scale_b * (A B^T), FP32 accumulation over all of K.
+
+    a: [M,K] E4M3; b: [N,K] E4M3; scale_a, scale_b: one-element fp32 device
+    tensors; d: [M,N] bf16 output.
+    """
+    M, K = a.shape
+    N = b.shape[0]
+    if scale_a.numel() != 1 or scale_b.numel() != 1:
+        raise ValueError("scale_a and scale_b hold one value each")
+    args = (_dev(a, "a", _FP8, 2), _dev(scale_a.reshape(1), "scale_a", _F32, 1),
+            _dev(b, "b", _FP8, 2), _dev(scale_b.reshape(1), "scale_b", _F32, 1),
+            _dev(d, "d", (torch.bfloat16,), 2))
+    if tuple(d.shape) != (M, N) or b.shape[1] != K:
+        raise ValueError("shape mismatch between a, b and d")
+    _check(load_library().gemm_fp8_fp8_bf16_nt_per_tensor(*args, M, N, K, _stream_ptr(stream)),
+           "gemm_fp8_fp8_bf16_nt_per_tensor")
     return d
 
 

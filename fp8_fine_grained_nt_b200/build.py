@@ -1,7 +1,7 @@
 """Build libfp8nt.so in-tree with nvcc for sm_100a (ahead of time, no JIT).
 
 Compiles csrc/api.cu and one object per kernel shape listed in
-csrc/kernels.def (csrc/instance.cu with -DFP8NT_MW / -DFP8NT_BN / -DFP8NT_PAIR), in
+csrc/kernels.def (csrc/instance.cu with -DFP8NT_MW / -DFP8NT_BN / -DFP8NT_PAIR / -DFP8NT_SCALAR), in
 parallel, then links them with the static CUDA runtime.  ptxas's resource
 report is checked for every kernel: the kernels rebalance registers between
 warpgroups with setmaxnreg, which is only safe when each kernel is launched
@@ -42,15 +42,26 @@ def nvcc() -> str:
     return cand
 
 
-def kernel_shapes() -> list[tuple[int, int, int]]:
-    """(MW, BN, PAIR) of every kernel listed in csrc/kernels.def."""
+def kernel_list() -> list[tuple[int, int, int, int]]:
+    """(MW, BN, PAIR, SCALAR) of every kernel listed in csrc/kernels.def."""
     shapes = []
     with open(os.path.join(CSRC, "kernels.def")) as f:
         for line in f:
-            m = re.match(r"\s*FP8NT_KERNEL\(\s*(\d+)\s*,\s*(\d+)\s*,\s*(\d+)\s*\)", line)
+            m = re.match(r"\s*FP8NT_KERNEL\(\s*(\d+)\s*,\s*(\d+)\s*,\s*(\d+)\s*,\s*(\d+)\s*\)",
+                         line)
             if m:
-                shapes.append((int(m.group(1)), int(m.group(2)), int(m.group(3))))
+                shapes.append(tuple(int(m.group(i)) for i in range(1, 5)))
     return shapes
+
+
+def kernel_shapes() -> list[tuple[int, int, int]]:
+    """(MW, BN, PAIR) of every fine-grained-scale kernel."""
+    return [(mw, bn, pair) for mw, bn, pair, scalar in kernel_list() if not scalar]
+
+
+def scalar_kernel_shapes() -> list[int]:
+    """BN of every per-tensor-scale kernel (MW = 1)."""
+    return [bn for mw, bn, pair, scalar in kernel_list() if scalar]
 
 
 def _sources_digest(extra: list[str]) -> str:
@@ -108,11 +119,11 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -
         return LIB_PATH
     jobs = jobs or max(1, os.cpu_count() or 1)
     tasks = [(os.path.join(CSRC, "api.cu"), os.path.join(BUILD_DIR, "api.o"), [], "api")]
-    for mw, bn, pair in kernel_shapes():
-        tasks.append((os.path.join(CSRC, "instance.cu"),
-                      os.path.join(BUILD_DIR, f"kernel_mw{mw}_bn{bn}_p{pair}.o"),
-                      [f"-DFP8NT_MW={mw}", f"-DFP8NT_BN={bn}", f"-DFP8NT_PAIR={pair}"],
-                      f"mw{mw}_bn{bn}_p{pair}"))
+    for mw, bn, pair, scalar in kernel_list():
+        tag = f"mw{mw}_bn{bn}_p{pair}_s{scalar}"
+        tasks.append((os.path.join(CSRC, "instance.cu"), os.path.join(BUILD_DIR, f"kernel_{tag}.o"),
+                      [f"-DFP8NT_MW={mw}", f"-DFP8NT_BN={bn}", f"-DFP8NT_PAIR={pair}",
+                       f"-DFP8NT_SCALAR={scalar}"], tag))
     notes = []
     with ThreadPoolExecutor(max_workers=jobs) as pool:
         futures = [(t, pool.submit(_compile, t[0], t[1], t[2])) for t in tasks]

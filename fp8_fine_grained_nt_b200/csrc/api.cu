@@ -22,12 +22,14 @@ namespace {
 struct Candidate {
     int mw;
     int bn;
-    int pair; // 1: a CTA pair computes a 256-row tile (tcgen05 cta_group::2)
+    int pair;   // 1: a CTA pair computes a 256-row tile (tcgen05 cta_group::2)
+    int scalar; // 1: per-tensor scaling (whole-K accumulation in TMEM)
     LaunchFn launch;
 };
 
 const Candidate kCandidates[] = {
-#define FP8NT_KERNEL(mw, bn, pair) {mw, bn, pair, launch_mw##mw##_bn##bn##_p##pair},
+#define FP8NT_KERNEL(mw, bn, pair, scalar)                                                       \
+    {mw, bn, pair, scalar, launch_mw##mw##_bn##bn##_p##pair##_s##scalar},
 #include "kernels.def"
 #undef FP8NT_KERNEL
 };
@@ -215,8 +217,10 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int split, int pair, i
     const int halves = (mw == 2 && rows_eff > 128) ? 2 : 1;
     const int kb_per_cta = ceil_div(nkb, split);
     const int cta_rows = pair ? 128 : (rows_eff < 128 * mw ? rows_eff : 128 * mw);
-    double tile = kb_per_cta * 1300.0 * kb_cost_factor(pair ? 1 : mw, bn, halves) + 1500.0 +
-                  3500.0 * bn * cta_rows / (256.0 * 128.0);
+    const double kb_cycles = pb.kind == DG_KIND_DENSE_PER_TENSOR
+                                 ? 4.0 * (bn / 2 > 64 ? bn / 2 : 64) + 150.0
+                                 : 1300.0 * kb_cost_factor(pair ? 1 : mw, bn, halves);
+    double tile = kb_per_cta * kb_cycles + 1500.0 + 3500.0 * bn * cta_rows / (256.0 * 128.0);
     if (split > 1)
         tile += 800.0 + (double)bm * bn * 4.0 * split / 256.0 / split;
     if (tiles_out)
@@ -271,6 +275,8 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
             continue;
         if (pb.kind == DG_KIND_CONTIGUOUS && c_bm != 128)
             continue; // a 256-row tile could straddle two 128-aligned experts
+        if ((pb.kind == DG_KIND_DENSE_PER_TENSOR) != (c.scalar != 0))
+            continue; // per-tensor and fine-grained scaling have their own kernels
         for (int split = 1; split <= kMaxSplit; split *= 2) {
             if (g_forced_split && split != g_forced_split)
                 continue;
@@ -335,7 +341,7 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
         cfg->grid = 1;
     cfg->smem_bytes = (int)plan->total + 1024;
     const int buf_cols = best->mw * best->bn;
-    const int nbuf = 512 / buf_cols < MAX_TMEM_BUFS ? 512 / buf_cols : MAX_TMEM_BUFS;
+    const int nbuf = best->scalar ? 2 : (512 / buf_cols < MAX_TMEM_BUFS ? 512 / buf_cols : MAX_TMEM_BUFS);
     const int need = nbuf * buf_cols; // the kernel's ring of K-block partials
     cfg->tmem_cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
     *out_cand = best;
@@ -386,7 +392,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
 
     const int nkb = pb.K / 128;
     const int nnb = ceil_div(pb.N, 128);
-    const int groups = pb.kind == DG_KIND_DENSE ? 1 : pb.groups;
+    const int groups = (pb.kind == DG_KIND_DENSE || pb.kind == DG_KIND_DENSE_PER_TENSOR) ? 1 : pb.groups;
     const int ld_sa = get_tma_aligned_size(pb.M, 4);
 
     CUtensorMap tmap_a, tmap_b, tmap_sa, tmap_d;
@@ -406,7 +412,9 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     // SA_SLOT_BYTES / (rows * 4) consecutive K blocks
     const long sa_groups = pb.kind == DG_KIND_MASKED ? groups : 1;
     const uint32_t sa_box_rows = cand->pair ? 128u : (uint32_t)cfg.block_m;
-    if ((st = make_tmap_2d(&tmap_sa, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)ld_sa,
+    memset(&tmap_sa, 0, sizeof(tmap_sa)); // per-tensor scaling: not read by the kernel
+    if (!cand->scalar &&
+        (st = make_tmap_2d(&tmap_sa, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)ld_sa,
                            (uint64_t)sa_groups * nkb, (uint64_t)ld_sa, sa_box_rows,
                            SA_SLOT_BYTES / (sa_box_rows * 4u), CU_TENSOR_MAP_SWIZZLE_NONE)) != DG_OK)
         return st;
@@ -419,7 +427,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
 
     Params p;
     memset(&p, 0, sizeof(p));
-    p.kind = pb.kind;
+    p.kind = pb.kind == DG_KIND_DENSE_PER_TENSOR ? DG_KIND_DENSE : pb.kind;
     p.M = pb.M;
     p.N = pb.N;
     p.K = pb.K;
@@ -469,6 +477,17 @@ int gemm_fp8_fp8_bf16_nt(const void *A, const float *sa, const void *B, const fl
         return st;
     Problem pb{DG_KIND_DENSE, M, N, K, 1, 0};
     return run(pb, A, sa, B, sb, D, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gemm_fp8_fp8_bf16_nt_per_tensor(const void *A, const float *scale_a, const void *B,
+                                    const float *scale_b, void *D, int M, int N, int K,
+                                    dg_stream_t stream)
+{
+    int st = check_common(A, scale_a, B, scale_b, D, M, N, K);
+    if (st != DG_OK || M == 0 || N == 0)
+        return st;
+    Problem pb{DG_KIND_DENSE_PER_TENSOR, M, N, K, 1, 0};
+    return run(pb, A, scale_a, B, scale_b, D, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *A, const float *sa, const void *B,
@@ -586,14 +605,15 @@ int dg_get_device_status(dg_stream_t stream)
 int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected_m, int num_sms,
                      dg_config *out)
 {
-    if (!out || kind < 0 || kind > 2 || M <= 0 || N <= 0 || K <= 0 || num_groups <= 0)
+    if (!out || kind < 0 || kind > 3 || M <= 0 || N <= 0 || K <= 0 || num_groups <= 0)
         return DG_ERR_INVALID_ARGUMENT;
     if (K % 128 != 0 || N % 8 != 0)
         return DG_ERR_UNSUPPORTED_SHAPE;
     if (kind == DG_KIND_MASKED && num_groups > MAX_MASKED_GROUPS)
         return DG_ERR_UNSUPPORTED_SHAPE;
     int sms = num_sms > 0 ? num_sms : (g_num_sms_limit > 0 ? g_num_sms_limit : kDefaultSms);
-    Problem pb{kind, M, N, K, kind == DG_KIND_DENSE ? 1 : num_groups, expected_m};
+    const bool one_group = kind == DG_KIND_DENSE || kind == DG_KIND_DENSE_PER_TENSOR;
+    Problem pb{kind, M, N, K, one_group ? 1 : num_groups, expected_m};
     const Candidate *cand = nullptr;
     SmemPlan plan;
     return choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);

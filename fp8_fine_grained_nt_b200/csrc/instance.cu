@@ -1,6 +1,6 @@
-// One (MW, BN, PAIR) instantiation of the GEMM kernel and its launcher; the
-// build compiles this file once per entry of kernels.def with -DFP8NT_MW,
-// -DFP8NT_BN and -DFP8NT_PAIR.
+// One (MW, BN, PAIR, SCALAR) instantiation of the GEMM kernel and its
+// launcher; the build compiles this file once per entry of kernels.def with
+// -DFP8NT_MW, -DFP8NT_BN, -DFP8NT_PAIR and -DFP8NT_SCALAR.
 #include <cuda_runtime.h>
 
 #include "kernel.cuh"
@@ -15,15 +15,18 @@
 #ifndef FP8NT_PAIR
 #error "FP8NT_PAIR must be defined"
 #endif
+#ifndef FP8NT_SCALAR
+#error "FP8NT_SCALAR must be defined"
+#endif
 
 namespace fp8nt {
 
-#define FP8NT_CAT_(a, b, c) launch_mw##a##_bn##b##_p##c
-#define FP8NT_NAME(a, b, c) FP8NT_CAT_(a, b, c)
+#define FP8NT_CAT_(a, b, c, d) launch_mw##a##_bn##b##_p##c##_s##d
+#define FP8NT_NAME(a, b, c, d) FP8NT_CAT_(a, b, c, d)
 
-cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN, FP8NT_PAIR)(const LaunchArgs &args)
+cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN, FP8NT_PAIR, FP8NT_SCALAR)(const LaunchArgs &args)
 {
-    auto kernel = fp8_gemm_kernel<FP8NT_MW, FP8NT_BN, FP8NT_PAIR != 0>;
+    auto kernel = fp8_gemm_kernel<FP8NT_MW, FP8NT_BN, FP8NT_PAIR != 0, FP8NT_SCALAR != 0>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            args.smem_bytes);
     if (err != cudaSuccess)

@@ -35,7 +35,7 @@
 
 namespace fp8nt {
 
-template <int MW, int BN, bool PAIR = false>
+template <int MW, int BN, bool PAIR = false, bool SCALAR = false>
 struct KernelTraits {
     static_assert(MW == 1 || MW == 2, "MW is 1 or 2");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be a multiple of 16 in [16, 256]");
@@ -52,7 +52,10 @@ struct KernelTraits {
     static constexpr int OUT_CHUNKS = ((MW == 1 ? BN / 2 : BN) + 31) / 32;
     static constexpr int BUF_COLS = MW * BN;                 // TMEM columns per K-block buffer
     // ring of K-block partial buffers in TMEM: as many as fit, at most 16
-    static constexpr int NBUF = (512 / BUF_COLS) < MAX_TMEM_BUFS ? (512 / BUF_COLS) : MAX_TMEM_BUFS;
+    // (SCALAR: one whole-K accumulator per tile, two tiles in flight)
+    static constexpr int NBUF = SCALAR ? 2
+                              : (512 / BUF_COLS) < MAX_TMEM_BUFS ? (512 / BUF_COLS) : MAX_TMEM_BUFS;
+    static_assert(!SCALAR || (MW == 1 && !PAIR), "per-tensor scaling uses one 128-row CTA per tile");
     static constexpr int TMEM_NEED = NBUF * BUF_COLS;
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                    : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
@@ -300,14 +303,14 @@ __device__ __forceinline__ void fma_range_any(float (&acc)[NC], const float (&v)
         fma_range<NC, C0, N, false>(acc, v, s_lo, s_hi, t);
 }
 
-template <int MW, int BN, bool PAIR>
+template <int MW, int BN, bool PAIR, bool SCALAR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_sa,
                     const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ Params p)
 {
-    using T = KernelTraits<MW, BN, PAIR>;
+    using T = KernelTraits<MW, BN, PAIR, SCALAR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -330,6 +333,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t *sa_full = sb_empty + 2;  // LHS-scale ring (2 slots)
     uint64_t *sa_empty = sa_full + 2;
     uint64_t *mma_done = sa_empty + 2;
+    uint64_t *tile_full = mma_done + 1; // per-tensor scaling: a tile's accumulator is complete (x2)
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + plan.off_misc);
     volatile uint32_t *abort_flag = misc + 1;
     int *prefix = reinterpret_cast<int *>(smem + plan.off_prefix);
@@ -354,13 +358,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&sa_empty[b], NUM_EPI_WARPS);
         }
         mbar_init(mma_done, 1);
+        mbar_init(&tile_full[0], 1);
+        mbar_init(&tile_full[1], 1);
         misc[1] = 0u;
         fence_mbarrier_init();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
-        tma_prefetch_desc(&tmap_sa);
+        if (!SCALAR)
+            tma_prefetch_desc(&tmap_sa);
         tma_prefetch_desc(&tmap_d);
     }
     if (warp == 1) {
@@ -413,7 +420,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Split-K: the p.split CTAs of a cluster share one output tile, each
     // computing K blocks [kb_lo, kb_hi); otherwise CTAs are persistent over
     // tiles and cover all K blocks.
-    const bool split_k = !PAIR && p.split > 1;
+    const bool split_k = !PAIR && !SCALAR && p.split > 1;
     const int split_rank = split_k ? (int)cluster_ctarank() : 0;
     // a CTA pair walks the pair tiles together; rank 0 is the leader
     const int pair_rank = PAIR ? (int)cluster_ctarank() : 0;
@@ -494,7 +501,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t stage_step = plan.stage_bytes >> 4;
             uint32_t kb_it = 0, s = 0, phase = 0;
             bool ok = true;
-            for (int t = t_first; ok && t < num_tiles; t += t_stride) {
+            if constexpr (SCALAR) {
+                // Per-tensor scaling: the tile's whole K range accumulates in
+                // TMEM buffer (tile mod 2); one commit per K block frees its
+                // stage, one more at the last K block publishes the tile.
+                uint32_t tile_it = 0;
+                for (int t = t_first; ok && t < num_tiles; t += t_stride) {
+                    const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+                    if (!ti.valid)
+                        continue;
+                    const uint32_t buf = tile_it & 1;
+                    if (!wait_bar(&tmem_empty[buf], ((tile_it >> 1) & 1) ^ 1, abort_flag, p))
+                        break;
+                    const uint32_t d = tmem_base + buf * (uint32_t)BN;
+                    for (int kb = kb_lo; kb < kb_hi; ++kb) {
+                        if (!wait_bar(&full[s], phase, abort_flag, p)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t a_desc = a_desc0 + s * stage_step;
+                        const uint64_t b_desc = b_desc0 + s * stage_step;
+#pragma unroll
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
+                            mma_f8f6f4(d, a_desc + (uint64_t)((k * MMA_K) >> 4),
+                                       b_desc + (uint64_t)((k * MMA_K) >> 4), idesc,
+                                       (kb > kb_lo || k > 0) ? 1u : 0u);
+                        mma_commit(&done[kb_it % DONE_RING]);
+                        if (kb == kb_hi - 1)
+                            mma_commit(&tile_full[buf]);
+                        ++kb_it;
+                        if (++s == (uint32_t)stages) {
+                            s = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    ++tile_it;
+                }
+            }
+            for (int t = t_first; !SCALAR && ok && t < num_tiles; t += t_stride) {
                 const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
                 if (!ti.valid)
                     continue;
@@ -555,6 +600,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 mma_commit(mma_done);
             wait_drain(mma_done, 0, abort_flag, p);
         }
+    } else if (warp == 3 && SCALAR) {
+        regs_dec<REGS_PRODUCER>(); // per-tensor scaling: no scale tiles to load
     } else if (warp == 3) {
         // ------------------------------------------------------------ scales
         // Per tile, the RHS scales (<= 3 rows of K/128 floats, cp.async by
@@ -622,12 +669,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
             if (!ti.valid)
                 continue;
+            const bool active = (MW == 1) ? true : (half * HALF_M < ti.rows);
+            const int cbase = ti.n0 + col0;
+            float acc[NC];
+            if constexpr (SCALAR) {
+                // Per-tensor scaling: read the tile's accumulator once, scale
+                // it by scale_a * scale_b, hand the buffer back.
+                const uint32_t buf = tile_it & 1;
+                if (!wait_bar_warp(&tile_full[buf], (tile_it >> 1) & 1, abort_flag, p))
+                    break;
+                tc_fence_after();
+                const float scale = __ldg(p.sa) * __ldg(p.sb);
+                const uint32_t taddr = tmem_base + lane_off + buf * (uint32_t)BN + (uint32_t)col0;
+                static_assert(NC % 32 == 0, "per-tensor tiles load 32-column chunks");
+#pragma unroll
+                for (int c = 0; c < NC; c += 32) {
+                    float(&v)[32] = *reinterpret_cast<float(*)[32]>(&acc[c]);
+                    tmem_ld32(taddr + c, v);
+                    tmem_wait_ld(v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        v[j] *= scale;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&tmem_empty[buf]);
+                ++tile_it;
+            } else {
             const int slot = tile_it & 1;
             if (!wait_bar_warp(&sb_full[slot], (tile_it >> 1) & 1, abort_flag, p))
                 break;
             const float *sbt = sb_tile + slot * MAX_SB_BLOCKS * pitch;
-            const bool active = (MW == 1) ? true : (half * HALF_M < ti.rows);
-            const int cbase = ti.n0 + col0;
             // scale blocks of this thread's columns: lo = block of its first
             // column (relative to the tile's first block), t_split = local
             // column where the next block starts
@@ -654,7 +727,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 s_lo = sa_v * sbt[lo * pitch + kb];
                 s_hi = sa_v * sbt[(lo + 1) * pitch + kb];
             };
-            float acc[NC];
 #pragma unroll
             for (int c = 0; c < NC; ++c)
                 acc[c] = 0.0f;
@@ -788,6 +860,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
                 continue;
             }
+            } // non-scalar promotion
 
             // ---- store the tile's rows as BF16
             bool row_ok = active && row_in_tile < ti.rows;

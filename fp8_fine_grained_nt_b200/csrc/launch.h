@@ -23,7 +23,8 @@ struct LaunchArgs {
 
 typedef cudaError_t (*LaunchFn)(const LaunchArgs &);
 
-#define FP8NT_KERNEL(mw, bn, pair) cudaError_t launch_mw##mw##_bn##bn##_p##pair(const LaunchArgs &);
+#define FP8NT_KERNEL(mw, bn, pair, scalar)                                                    \
+    cudaError_t launch_mw##mw##_bn##bn##_p##pair##_s##scalar(const LaunchArgs &);
 #include "kernels.def"
 #undef FP8NT_KERNEL
 

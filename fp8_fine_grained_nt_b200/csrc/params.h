@@ -106,8 +106,9 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     off = p.off_prefix + 4u * (uint32_t)prefix_ints;
     p.off_bars = align_up_u32(off, 8);
     // full per stage, the ring of "K block done" barriers, TMEM empty per
-    // partial buffer, sb and sa full/empty x2, one "all MMAs done" barrier
-    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u);
+    // partial buffer, sb and sa full/empty x2, one "all MMAs done" barrier,
+    // two "tile accumulated" barriers (per-tensor scaling)
+    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u + 2u);
     p.off_misc = align_up_u32(off, 16);
     p.total = p.off_misc + 16;
     return p;

@@ -67,6 +67,18 @@ typedef enum dg_status {
 int gemm_fp8_fp8_bf16_nt(const void *A, const float *sa, const void *B, const float *sb,
                          void *D, int M, int N, int K, dg_stream_t stream);
 
+/* Dense GEMM with per-tensor scaling (the tensor-wise FP8 recipe that the
+ * FP8-training blog page contrasts with fine-grained scaling, section 4.2):
+ *   D[m,n] = scale_a * scale_b * sum_k A[m,k] * B[n,k]
+ * accumulated in FP32 over the whole K range in tensor memory (no per-block
+ * promotion is needed when every block has the same scale) and rounded to
+ * BF16 (RNE).  scale_a and scale_b point to ONE FP32 value each, in device
+ * memory (read by the kernel, so a CUDA graph can update them).  A, B, D and
+ * the shape rules are as for gemm_fp8_fp8_bf16_nt. */
+int gemm_fp8_fp8_bf16_nt_per_tensor(const void *A, const float *scale_a, const void *B,
+                                    const float *scale_b, void *D, int M, int N, int K,
+                                    dg_stream_t stream);
+
 /* Contiguous m-grouped GEMM (DeepGEMM README, grouped GEMMs: tokens of all
  * experts concatenated into one tensor, each expert segment aligned to
  * get_m_alignment_for_contiguous_layout(); only the M axis is grouped, all
@@ -144,7 +156,7 @@ typedef struct dg_config {
                        of A and half of the B tile); 1: one CTA per tile */
 } dg_config;
 
-enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2 };
+enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2, DG_KIND_DENSE_PER_TENSOR = 3 };
 
 /* The configuration a call of `kind` would use.  For DG_KIND_DENSE: M, N, K;
  * for DG_KIND_CONTIGUOUS: M = M_sum; for DG_KIND_MASKED: M = M_max and

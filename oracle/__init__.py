@@ -191,6 +191,18 @@ def gemm_masked_sampled(*args, **kw):
     return default().gemm_masked_sampled(*args, **kw)
 
 
+def gemm_per_tensor(a, scale_a: float, b, scale_b: float, M: int, N: int, K: int,
+                    lib: OracleLib | None = None) -> np.ndarray:
+    """Per-tensor scaling (one FP32 scale per operand; the tensor-wise recipe
+    of the FP8-training blog page, section 4.2): the fine-grained definition
+    with every LHS and RHS block scale equal, i.e.
+    D = scale_a * scale_b * sum_k dec(A[m,k]) dec(B[n,k])."""
+    nkb = K // 128
+    sa = np.full((nkb, M), np.float32(scale_a), dtype=np.float32)
+    sb = np.full(((N + 127) // 128, nkb), np.float32(scale_b), dtype=np.float32)
+    return (lib or default()).gemm_dense(a, sa, b, sb, M, N, K)
+
+
 def num_threads() -> int:
     """Threads OpenMP will use for the oracle (OMP_NUM_THREADS, else all cores)."""
     env = os.environ.get("OMP_NUM_THREADS")

@@ -331,3 +331,64 @@ def test_full_size_masked(name):
     unt = H.untouched(d)
     for g in range(prob.G):
         assert unt[g, mm[g]:].all(), f"group {g}: rows beyond masked_m written"
+
+
+# --------------------------------------------------------------------- per-tensor scaling
+
+
+def run_per_tensor(a, scale_a, b, scale_b, M, N):
+    d = H.sentinel_like((M, N))
+    fp8.gemm_fp8_fp8_bf16_nt_per_tensor(a.cuda(), torch.tensor([scale_a], device="cuda"), b.cuda(),
+                                        torch.tensor([scale_b], device="cuda"), d)
+    torch.cuda.synchronize()
+    return d
+
+
+def per_tensor_problem(M, N, K, seed):
+    g = torch.Generator().manual_seed(seed)
+    a = torch.randn(M, K, generator=g).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    b = torch.randn(N, K, generator=g).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    return a, b
+
+
+def scalar_shapes():
+    from fp8_fine_grained_nt_b200 import build
+    return build.scalar_kernel_shapes()
+
+
+@pytest.mark.parametrize("bn", scalar_shapes())
+def test_per_tensor_every_kernel_shape(bn):
+    """Whole-K accumulation in TMEM, ragged M and N, several K blocks."""
+    M, N, K = 300, 400, 1280
+    a, b = per_tensor_problem(M, N, K, 500 + bn)
+    ref = oracle.gemm_per_tensor(a, 0.02, b, 0.5, M, N, K)
+    fp8.force_config(128, bn)
+    try:
+        d = run_per_tensor(a, 0.02, b, 0.5, M, N)
+    finally:
+        fp8.force_config(0, 0)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, f"per-tensor bn{bn}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 128), (129, 136, 7168), (512, 2112, 7168)])
+def test_per_tensor_auto_config(M, N, K):
+    a, b = per_tensor_problem(M, N, K, M + N + K)
+    ref = oracle.gemm_per_tensor(a, 0.125, b, 0.25, M, N, K)
+    d = run_per_tensor(a, 0.125, b, 0.25, M, N)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, f"per-tensor {M}x{N}x{K}")
+
+
+def test_per_tensor_full_size_sampled():
+    """4096 x 7168 x 2048 in the configuration the benchmark launches: sampled
+    rows against the oracle, and bit-identical repeats."""
+    M, N, K = 4096, 7168, 2048
+    a, b = per_tensor_problem(M, N, K, 77)
+    d1 = run_per_tensor(a, 0.01, b, 0.03, M, N)
+    d2 = run_per_tensor(a, 0.01, b, 0.03, M, N)
+    check_status()
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+    rows = np.random.default_rng(3).choice(M, 24, replace=False)
+    ref = oracle.gemm_per_tensor(a[rows].contiguous(), 0.01, b, 0.03, len(rows), N, K)
+    H.assert_close(H.bf16_bits_to_f64(d1)[rows], ref, "per-tensor full size")

@@ -222,3 +222,23 @@ def test_binding_rejects_cpu_tensors(lib):
     s = torch.zeros(1, 128, dtype=torch.float32)
     with pytest.raises((ValueError, TypeError)):
         fp8.gemm_fp8_fp8_bf16_nt(t, s, t, s, torch.zeros(128, 128, dtype=torch.bfloat16))
+
+
+def test_per_tensor_host_checks_and_selection(lib):
+    p = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10008)
+    g = lib.gemm_fp8_fp8_bf16_nt_per_tensor
+    assert g(p, p, p, p, p, 128, 128, 100, None) == 3   # K % 128
+    assert g(p, p, p, p, p, 128, 100, 128, None) == 3   # N % 8
+    assert g(p, p, p, p, p, 0, 128, 128, None) == 0     # empty
+    assert g(p, None, p, p, p, 128, 128, 128, None) == 1
+    assert g(p, p, mis, p, p, 128, 128, 128, None) == 2
+    from fp8_fine_grained_nt_b200 import build
+    scalar_bns = set(build.scalar_kernel_shapes())
+    assert scalar_bns and scalar_bns <= {64, 128, 192, 256}
+    for M, N, K in ((4096, 7168, 2048), (1, 8, 128), (300, 400, 512), (8192, 8192, 8192)):
+        cfg = fp8.select_config(fp8.KIND_DENSE_PER_TENSOR, M, N, K, num_sms=148)
+        assert cfg["block_m"] == 128 and cfg["block_n"] in scalar_bns
+        assert cfg["split"] == 1 and cfg["cta_pair"] == 1
+        assert cfg["tmem_cols"] >= 2 * cfg["block_n"]
+    assert fp8.select_config(fp8.KIND_DENSE_PER_TENSOR, 4096, 7168, 2048, num_sms=148)["block_n"] == 256

@@ -290,6 +290,20 @@ def pin_sampled_equal_full(lib):
     assert np.array_equal(msamp[~np.isnan(ref)], ref[~np.isnan(ref)])
 
 
+def pin_per_tensor_equals_scaled_library_matmul(lib):
+    """Per-tensor scaling is the special case of equal block scales: it must
+    equal scale_a * scale_b * (decoded A) @ (decoded B)^T, the partials being
+    exact in FP64 (any order)."""
+    rng = np.random.default_rng(11)
+    M, N, K = 37, 45, 640
+    a = random_finite_bytes(rng, (M, K))
+    b = random_finite_bytes(rng, (N, K))
+    sa_, sb_ = 0.0078125 * 3, 1.0 / 448.0
+    got = oracle.gemm_per_tensor(a, sa_, b, sb_, M, N, K, lib=lib)
+    ref = (torch_decode(a) @ torch_decode(b).T) * (np.float64(np.float32(sa_)) * np.float64(np.float32(sb_)))
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-9 * np.abs(ref).max())
+
+
 PINS = [
     pin_decode_table_matches_torch,
     pin_decode_golden_range,
@@ -305,6 +319,7 @@ PINS = [
     pin_masked_closed_form_and_untouched,
     pin_masked_equals_per_group_dense,
     pin_sampled_equal_full,
+    pin_per_tensor_equals_scaled_library_matmul,
 ]
 
 
