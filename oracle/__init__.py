@@ -55,6 +55,7 @@ class OracleLib:
             "oracle_gemm_contiguous_sampled": [P, P, L, P, P, P, I, I, I, I, P, P, L, P],
             "oracle_gemm_masked": [P, P, L, P, P, P, I, I, I, I, P],
             "oracle_gemm_masked_sampled": [P, P, L, P, P, P, I, I, I, I, P, P, P, L, P],
+            "oracle_quantize_1x128": [P, I, I, P, P, L],
         }
         for name, argtypes in sigs.items():
             fn = getattr(lib, name)
@@ -119,6 +120,18 @@ class OracleLib:
             _ptr(a), _ptr(sa), sa.shape[-1], _ptr(b), _ptr(sb), _ptr(mm), G, M_max, N, K,
             _ptr(out)), "gemm_masked")
         return out
+
+    def quantize_1x128(self, x, M: int, K: int, ld_sa: int | None = None):
+        """(q uint8 [M, K], sa float32 [K/128, ld_sa]) of an FP32 [M, K] input
+        (BF16 inputs: pass their exact FP32 values).  Columns M..ld_sa-1 of sa
+        are left NaN (not part of the definition)."""
+        x = _np(x, np.float32)
+        ld = ld_sa if ld_sa is not None else (M + 3) // 4 * 4
+        q = np.empty((M, K), dtype=np.uint8)
+        sa = np.full((K // 128, ld), np.nan, dtype=np.float32)
+        _check(self.lib.oracle_quantize_1x128(_ptr(x), M, K, _ptr(q), _ptr(sa), ld),
+               "quantize_1x128")
+        return q, sa
 
     def gemm_masked_sampled(self, a, sa, b, sb, masked_m, G, M_max, N, K, groups, rows,
                             cols) -> np.ndarray:
@@ -189,6 +202,10 @@ def gemm_masked(*args, **kw):
 
 def gemm_masked_sampled(*args, **kw):
     return default().gemm_masked_sampled(*args, **kw)
+
+
+def quantize_1x128(*args, **kw):
+    return default().quantize_1x128(*args, **kw)
 
 
 def gemm_per_tensor(a, scale_a: float, b, scale_b: float, M: int, N: int, K: int,

@@ -262,3 +262,77 @@ int oracle_gemm_masked_sampled(const uint8_t *A, const float *sa, long ld_sa, co
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * 1x128 activation quantiser (the step before the GEMM: the DeepGEMM README,
+ * usage, leaves the cast and the transposition of the LHS scales to a
+ * preceding kernel; the DeepSeek-V3 recipe cited above fixes the 1x128 tile).
+ *
+ * Reading (the pages give no formula): per row m and 128-wide K block kb,
+ *   amax = max |x[m,k]| over the block              (FP32, exact)
+ *   s    = max(amax, 1e-4) / 448                    (FP32 division, RN)
+ *   q    = E4M3( clamp(x / s, -448, 448) )          (FP32 division, RN;
+ *          round to nearest E4M3 value, ties to the even mantissa)
+ * so that x ~ dec(q) * s; s goes to sa[kb * ld_sa + m] (column-major).
+ * Inputs must be finite.
+ */
+
+/* Nearest E4M3 byte to a finite float in [-448, 448], ties to the even
+ * mantissa bit, by search over the decode table (no bit tricks). */
+static uint8_t e4m3_encode_nearest(float y, const double *dec)
+{
+    double v = (double)y;
+    uint8_t best = 0;
+    double best_err = INFINITY;
+    for (int code = 0; code < 256; ++code) {
+        double d = dec[code];
+        if (isnan(d))
+            continue;
+        /* zero is stored as +0 for a non-negative input and -0 otherwise */
+        if (d == 0.0 && (code == 0x80) != (signbit(y) != 0))
+            continue;
+        double err = fabs(d - v);
+        if (err < best_err || (err == best_err && (code & 1) == 0 && (best & 1) == 1)) {
+            best = (uint8_t)code;
+            best_err = err;
+        }
+    }
+    return best;
+}
+
+int oracle_quantize_1x128(const float *x, int M, int K, uint8_t *q, float *sa, long ld_sa)
+{
+    if (M < 0 || K <= 0 || K % ORACLE_BLOCK != 0 || ld_sa < M)
+        return 1;
+    double dec[256];
+    oracle_e4m3_table(dec);
+    const int nkb = K / ORACLE_BLOCK;
+    const float floor_amax = 1e-4f;
+    const float e4m3_max = 448.0f;
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; ++m) {
+        for (int kb = 0; kb < nkb; ++kb) {
+            const float *xb = x + (long)m * K + (long)kb * ORACLE_BLOCK;
+            float amax = 0.0f;
+            for (int k = 0; k < ORACLE_BLOCK; ++k) {
+                float a = fabsf(xb[k]);
+                if (a > amax)
+                    amax = a;
+            }
+            if (amax < floor_amax)
+                amax = floor_amax;
+            volatile float s = amax / e4m3_max; /* one FP32 rounding */
+            for (int k = 0; k < ORACLE_BLOCK; ++k) {
+                volatile float y = xb[k] / s;
+                float yc = y;
+                if (yc > e4m3_max)
+                    yc = e4m3_max;
+                if (yc < -e4m3_max)
+                    yc = -e4m3_max;
+                q[(long)m * K + (long)kb * ORACLE_BLOCK + k] = e4m3_encode_nearest(yc, dec);
+            }
+            sa[(long)kb * ld_sa + m] = s;
+        }
+    }
+    return 0;
+}

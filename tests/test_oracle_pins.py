@@ -304,6 +304,76 @@ def pin_per_tensor_equals_scaled_library_matmul(lib):
     assert np.allclose(got, ref, rtol=1e-12, atol=1e-9 * np.abs(ref).max())
 
 
+def pin_quantize_exact_blocks(lib):
+    """Blocks whose amax is 448 * 2^j hold values dec(code) * 2^j: the scale
+    must be exactly 2^j and every code must come back unchanged; a zero
+    block gets the amax floor (1e-4 / 448 in FP32) and zero codes; the block
+    maximum lands on +-448."""
+    rng = np.random.default_rng(5)
+    M, K = 6, 384
+    codes = random_finite_bytes(rng, (M, K))
+    codes[codes == 0x80] = 0x00              # -0 encodes as +0 after scaling
+    x = np.empty((M, K), dtype=np.float32)
+    exps = [-3, 0, 5]
+    for kb in range(K // 128):
+        blk = codes[:, kb * 128:(kb + 1) * 128]
+        blk[:, 7] = 0x7E                     # each row's amax is exactly 448
+        x[:, kb * 128:(kb + 1) * 128] = torch_decode(blk) * 2.0 ** exps[kb]
+    x[5, 128:256] = 0.0
+    q, sa = lib.quantize_1x128(x, M, K)
+    expect_q = codes.copy()
+    expect_q[5, 128:256] = 0
+    assert np.array_equal(q, expect_q)
+    for kb in range(K // 128):
+        want = np.full(M, np.float32(2.0 ** exps[kb]), dtype=np.float32)
+        if kb == 1:
+            want[5] = np.float32(np.float32(1e-4) / np.float32(448.0))
+        assert np.array_equal(sa[kb, :M], want), kb
+
+
+def pin_quantize_ties_to_even(lib):
+    """With a unit scale (amax 448), values halfway between two E4M3 values
+    go to the even mantissa: 1.0625 -> 1.0 (0x38), 1.1875 -> 1.25 (0x3A),
+    -1.0625 -> -1.0 (0xB8); 0.0009765625 (half of the smallest subnormal)
+    -> 0."""
+    x = np.zeros((1, 128), dtype=np.float32)
+    x[0, :5] = [448.0, 1.0625, 1.1875, -1.0625, 0.0009765625]
+    q, sa = lib.quantize_1x128(x, 1, 128)
+    assert sa[0, 0] == 1.0
+    assert q[0, :5].tolist() == [0x7E, 0x38, 0x3A, 0xB8, 0x00]
+
+
+def pin_quantize_unit_scale_equals_library_cast(lib):
+    """With a unit scale the quantiser is a plain round-to-nearest-even cast,
+    which torch's float8_e4m3fn conversion (a library routine) performs."""
+    rng = np.random.default_rng(9)
+    x = rng.uniform(-448, 448, size=(4, 256)).astype(np.float32)
+    x[:, 0] = 448.0
+    x[:, 128] = -448.0
+    q, sa = lib.quantize_1x128(x, 4, 256)
+    assert np.all(sa[:, :4] == 1.0)
+    ref = torch.from_numpy(x).to(E4M3).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+
+
+def pin_quantize_round_trip_bound(lib):
+    """For N(0,1) data: dec(q) * s is within half an E4M3 step of x (relative
+    2^-4 for normal values, absolute 2^-10 * s below), signs agree, and the
+    scale is amax / 448 to within one FP32 rounding."""
+    rng = np.random.default_rng(13)
+    M, K = 33, 512
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    q, sa = lib.quantize_1x128(x, M, K)
+    s = np.repeat(sa[:, :M].T, 128, axis=1).astype(np.float64)
+    back = torch_decode(q) * s
+    err = np.abs(back - x)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, s * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    assert np.all((np.sign(back) == np.sign(x)) | (back == 0))
+    amax = np.abs(x.reshape(M, K // 128, 128)).max(axis=2)
+    assert np.allclose(sa[:, :M].T, amax / 448.0, rtol=2.0 ** -23, atol=0)
+
+
 PINS = [
     pin_decode_table_matches_torch,
     pin_decode_golden_range,
@@ -320,6 +390,10 @@ PINS = [
     pin_masked_equals_per_group_dense,
     pin_sampled_equal_full,
     pin_per_tensor_equals_scaled_library_matmul,
+    pin_quantize_exact_blocks,
+    pin_quantize_ties_to_even,
+    pin_quantize_unit_scale_equals_library_cast,
+    pin_quantize_round_trip_bound,
 ]
 
 
@@ -362,6 +436,13 @@ MUTANTS = {
                                "const float *sag = sa;"),
     "masked_row_bound": ("if (m >= masked_m[g]) {\n                for",
                          "if (m > masked_m[g]) {\n                for"),
+    "quant_ties_away": ("(err == best_err && (code & 1) == 0 && (best & 1) == 1)",
+                        "(err == best_err && fabs(d) > fabs(dec[best]))"),
+    "quant_no_floor": ("if (amax < floor_amax)\n                amax = floor_amax;",
+                       "if (amax < 0.0f)\n                amax = floor_amax;"),
+    "quant_amax_signed": ("float a = fabsf(xb[k]);", "float a = xb[k];"),
+    "quant_scale_row_major": ("sa[(long)kb * ld_sa + m] = s;", "sa[(long)m * nkb + kb] = s;"),
+    "quant_scale_448_off": ("const float e4m3_max = 448.0f;", "const float e4m3_max = 440.0f;"),
 }
 
 
