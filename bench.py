@@ -337,6 +337,60 @@ def run_reference(args):
     return 0
 
 
+def measure_next_rows(fp8, peaks, iters: int = 20) -> dict:
+    """The rows built beyond the fine-grained GEMM, each timed alone (CUDA
+    events around every call, L2 flushed before each): the 1x128 activation
+    quantiser and the per-tensor-scale GEMM."""
+    dev = "cuda"
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn) -> float:
+        for _ in range(3):
+            fn()
+        total = 0.0
+        for _ in range(iters):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            total += e0.elapsed_time(e1)
+        return total / iters * 1e-3
+
+    out = {}
+    g = torch.Generator(device=dev).manual_seed(99)
+    M, K = 4096, 7168
+    ld = fp8.get_tma_aligned_size(M, 4)
+    q = torch.empty(M, K, dtype=torch.uint8, device=dev)
+    sa = torch.empty(K // 128, ld, dtype=torch.float32, device=dev)
+    for name, dt, esz in (("fp32", torch.float32, 4), ("bf16", torch.bfloat16, 2)):
+        x = torch.randn(M, K, generator=g, device=dev).to(dt)
+        t = timed(lambda: fp8.quantize_fp8_1x128(x, q, sa))
+        nbytes = esz * M * K + M * K + 4 * M * (K // 128)
+        out[f"quantize_1x128_{name}_{M}x{K}"] = {
+            "us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1), "bytes": nbytes,
+            "bound": "hbm", "roofline_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4)}
+        del x
+    M, N, K = 4096, 7168, 2048
+    a = torch.randint(0, 0x7E, (M, K), generator=g, device=dev, dtype=torch.uint8)
+    b = torch.randint(0, 0x7E, (N, K), generator=g, device=dev, dtype=torch.uint8)
+    sa1 = torch.tensor([0.01], device=dev)
+    sb1 = torch.tensor([0.02], device=dev)
+    d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    t = timed(lambda: fp8.gemm_fp8_fp8_bf16_nt_per_tensor(a, sa1, b, sb1, d))
+    flop = 2 * M * N * K
+    peak = 2.0 * peaks["bf16_tflops"]
+    out[f"per_tensor_gemm_{M}x{N}x{K}"] = {
+        "us": round(t * 1e6, 2), "tflops": round(flop / t / 1e12, 1), "flop": flop,
+        "bound": "tensor", "roofline_frac": round(flop / t / 1e12 / peak, 4)}
+    status = fp8.get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the extra rows: {fp8.status_string(status)}")
+    return out
+
+
 def run_gpu(args):
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -448,6 +502,8 @@ def run_gpu(args):
         unit = "GB/s"
     traffic = profiled_traffic(dom.name)
 
+    next_rows = measure_next_rows(fp8, peaks) if (rank == 0 and not args.no_next_rows) else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_sample(cases, args.cpu_budget_s)
@@ -478,6 +534,7 @@ def run_gpu(args):
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": len(cases) * args.steps,
             "clocks": clock_info,
+            "next_rows": next_rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -496,6 +553,8 @@ def main():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip timing the quantiser and the per-tensor GEMM")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -22,6 +22,7 @@ __all__ = [
     "load_library",
     "gemm_fp8_fp8_bf16_nt",
     "gemm_fp8_fp8_bf16_nt_per_tensor",
+    "quantize_fp8_1x128",
     "m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
     "m_grouped_gemm_fp8_fp8_bf16_nt_masked",
     "get_m_alignment_for_contiguous_layout",
@@ -82,6 +83,7 @@ def load_library():
         P, I = ctypes.c_void_p, ctypes.c_int
         lib.gemm_fp8_fp8_bf16_nt.argtypes = [P, P, P, P, P, I, I, I, P]
         lib.gemm_fp8_fp8_bf16_nt_per_tensor.argtypes = [P, P, P, P, P, I, I, I, P]
+        lib.quantize_fp8_1x128.argtypes = [P, I, P, P, I, I, P]
         lib.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         lib.m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.get_m_alignment_for_contiguous_layout.argtypes = []
@@ -171,6 +173,23 @@ def gemm_fp8_fp8_bf16_nt_per_tensor(a: torch.Tensor, scale_a: torch.Tensor, b: t
     _check(load_library().gemm_fp8_fp8_bf16_nt_per_tensor(*args, M, N, K, _stream_ptr(stream)),
            "gemm_fp8_fp8_bf16_nt_per_tensor")
     return d
+
+
+def quantize_fp8_1x128(x: torch.Tensor, q: torch.Tensor, sa: torch.Tensor,
+                       stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """1x128 quantiser: x [M,K] fp32 or bf16 -> q [M,K] E4M3 (uint8 or
+    float8_e4m3fn) and sa [K/128, get_tma_aligned_size(M, 4)] fp32 column-major."""
+    M, K = x.shape
+    dtype = {torch.float32: 0, torch.bfloat16: 1}.get(x.dtype)
+    if dtype is None:
+        raise TypeError(f"x has dtype {x.dtype}, expected float32 or bfloat16")
+    args = (_dev(x, "x", (torch.float32, torch.bfloat16), 2), dtype, _dev(q, "q", _FP8, 2),
+            _dev(sa, "sa", _F32, 2))
+    if tuple(q.shape) != (M, K) or sa.shape[0] != K // 128 or sa.shape[1] != get_tma_aligned_size(M, 4):
+        raise ValueError("shape mismatch between x, q and sa")
+    _check(load_library().quantize_fp8_1x128(*args, M, K, _stream_ptr(stream)),
+           "quantize_fp8_1x128")
+    return q, sa
 
 
 def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(a, sa, b, sb, d, m_indices, stream=None):

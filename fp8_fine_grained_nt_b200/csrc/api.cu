@@ -534,6 +534,30 @@ int m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *A, const float *sa, const 
     return run(pb, A, sa, B, sb, D, nullptr, masked_m, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int quantize_fp8_1x128(const void *x, int x_dtype, void *q, float *sa, int M, int K,
+                       dg_stream_t stream)
+{
+    if (M < 0 || K < 0 || (x_dtype != DG_INPUT_F32 && x_dtype != DG_INPUT_BF16))
+        return DG_ERR_INVALID_ARGUMENT;
+    if (K == 0 || K % 128 != 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0)
+        return DG_OK;
+    if (!x || !q || !sa)
+        return DG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sa))
+        return DG_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = device_info(&dev);
+    if (st != DG_OK)
+        return st;
+    const long ld_sa = get_tma_aligned_size(M, 4);
+    return launch_quantize_1x128(x, x_dtype == DG_INPUT_BF16, static_cast<uint8_t *>(q), sa, M, K,
+                                 ld_sa, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DG_OK
+               : DG_ERR_CUDA;
+}
+
 int get_m_alignment_for_contiguous_layout(void) { return 128; }
 
 int get_tma_aligned_size(int x, int element_size)

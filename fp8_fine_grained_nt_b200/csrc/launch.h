@@ -23,6 +23,10 @@ struct LaunchArgs {
 
 typedef cudaError_t (*LaunchFn)(const LaunchArgs &);
 
+// 1x128 activation quantiser (csrc/quantize.cu).
+cudaError_t launch_quantize_1x128(const void *x, bool bf16_in, uint8_t *q, float *sa, int M, int K,
+                                  long ld_sa, cudaStream_t stream);
+
 #define FP8NT_KERNEL(mw, bn, pair, scalar)                                                    \
     cudaError_t launch_mw##mw##_bn##bn##_p##pair##_s##scalar(const LaunchArgs &);
 #include "kernels.def"

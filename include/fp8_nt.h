@@ -115,6 +115,22 @@ int m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *A, const float *sa, const 
                                           int M_max, int N, int K, int expected_m,
                                           dg_stream_t stream);
 
+/* 1x128 activation quantiser: the cast and LHS-scale transposition that the
+ * DeepGEMM README (usage) leaves to a kernel before the GEMM; 1x128 tiles as
+ * in the DeepSeek-V3 recipe cited above.  For each row m and 128-wide K block
+ * kb of x [M,K] (row-major; FP32 or BF16 by x_dtype):
+ *   s = max(max_k |x[m,k]|, 1e-4) / 448              (FP32, IEEE division)
+ *   q[m,k] = E4M3(clamp(x[m,k] / s, -448, 448))      (IEEE division, then
+ *                                                      round to nearest even)
+ * q is [M,K] E4M3 bytes (row-major); s goes to sa[kb * ld + m] with
+ * ld = get_tma_aligned_size(M, 4): the column-major layout every GEMM entry
+ * point reads (columns M..ld-1 are not written).  x must be finite.
+ * K % 128 == 0; pointers 16-byte aligned device memory owned by the caller;
+ * M == 0 does nothing. */
+enum { DG_INPUT_F32 = 0, DG_INPUT_BF16 = 1 };
+int quantize_fp8_1x128(const void *x, int x_dtype, void *q, float *sa, int M, int K,
+                       dg_stream_t stream);
+
 /* Row alignment of each expert segment in the contiguous layout (DeepGEMM
  * README, utility functions: get_m_alignment_for_contiguous_layout).  128. */
 int get_m_alignment_for_contiguous_layout(void);

@@ -392,3 +392,71 @@ def test_per_tensor_full_size_sampled():
     rows = np.random.default_rng(3).choice(M, 24, replace=False)
     ref = oracle.gemm_per_tensor(a[rows].contiguous(), 0.01, b, 0.03, len(rows), N, K)
     H.assert_close(H.bf16_bits_to_f64(d1)[rows], ref, "per-tensor full size")
+
+
+# --------------------------------------------------------------------- quantiser (1x128)
+
+
+def run_quantize(x: torch.Tensor):
+    M, K = x.shape
+    ld = inputs.tma_aligned_size(M, 4)
+    q = torch.full((M, K), 0xAA, dtype=torch.uint8, device="cuda")
+    sa = torch.full((K // 128, ld), float("nan"), dtype=torch.float32, device="cuda")
+    fp8.quantize_fp8_1x128(x.cuda(), q, sa)
+    torch.cuda.synchronize()
+    check_status()
+    return q.cpu().numpy(), sa.cpu().numpy()
+
+
+def assert_quant_equal(x32: np.ndarray, q, sa, what):
+    M, K = x32.shape
+    q_ref, sa_ref = oracle.quantize_1x128(x32, M, K, ld_sa=sa.shape[1])
+    assert np.array_equal(q, q_ref), f"{what}: {int((q != q_ref).sum())} codes differ"
+    assert np.array_equal(sa[:, :M], sa_ref[:, :M]), f"{what}: scales differ"
+    assert np.isnan(sa[:, M:]).all(), f"{what}: padding columns written"
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (31, 256), (300, 1280), (64, 7168)])
+def test_quantize_fp32_bit_exact(M, K):
+    g = torch.Generator().manual_seed(M * 131 + K)
+    x = torch.randn(M, K, generator=g) * torch.exp(torch.randn(M, 1, generator=g) * 3)
+    q, sa = run_quantize(x)
+    assert_quant_equal(x.numpy(), q, sa, f"fp32 {M}x{K}")
+
+
+def test_quantize_bf16_bit_exact():
+    g = torch.Generator().manual_seed(7)
+    x = (torch.randn(257, 1024, generator=g) * 5).to(torch.bfloat16)
+    q, sa = run_quantize(x)
+    assert_quant_equal(x.float().numpy(), q, sa, "bf16")
+
+
+def test_quantize_edge_values():
+    """Zero blocks (amax floor), -0, huge and tiny magnitudes, exact maxima."""
+    x = torch.zeros(40, 512)
+    x[1, :128] = -0.0
+    x[2, 128:256] = 1e30
+    x[2, 130] = -3e30
+    x[3, 256:384] = 1e-30
+    x[4, :] = torch.linspace(-448, 448, 512)
+    x[5, 384:] = torch.tensor([1.0625, 1.1875, -1.0625] * 42 + [448.0, -448.0])
+    q, sa = run_quantize(x)
+    assert_quant_equal(x.numpy(), q, sa, "edges")
+
+
+def test_quantize_full_size_then_gemm():
+    """4096 x 7168 activations quantised on the device match the oracle
+    bit for bit, and feed the GEMM directly."""
+    M, K, N = 4096, 7168, 256
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn(M, K, generator=g)
+    q, sa = run_quantize(x)
+    assert_quant_equal(x.numpy(), q, sa, "full size")
+    prob = inputs.make_dense(M, N, K, seed=22)
+    d = H.sentinel_like((M, N))
+    fp8.gemm_fp8_fp8_bf16_nt(torch.from_numpy(q).cuda(), torch.from_numpy(sa).cuda(), prob.b.cuda(),
+                             prob.sb.cuda(), d)
+    torch.cuda.synchronize()
+    rows = np.arange(0, M, 97)
+    ref = oracle.gemm_dense(q[rows], sa[:, rows].copy(), prob.b, prob.sb, len(rows), N, K)
+    H.assert_close(H.bf16_bits_to_f64(d)[rows], ref, "quantised then GEMM")

@@ -242,3 +242,16 @@ def test_per_tensor_host_checks_and_selection(lib):
         assert cfg["split"] == 1 and cfg["cta_pair"] == 1
         assert cfg["tmem_cols"] >= 2 * cfg["block_n"]
     assert fp8.select_config(fp8.KIND_DENSE_PER_TENSOR, 4096, 7168, 2048, num_sms=148)["block_n"] == 256
+
+
+def test_quantize_host_checks(lib):
+    p = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10008)
+    qz = lib.quantize_fp8_1x128
+    assert qz(p, 0, p, p, 128, 100, None) == 3   # K % 128
+    assert qz(p, 0, p, p, 128, 0, None) == 3
+    assert qz(p, 2, p, p, 128, 128, None) == 1   # unknown input type
+    assert qz(p, 0, p, p, -1, 128, None) == 1
+    assert qz(p, 0, p, p, 0, 128, None) == 0     # empty
+    assert qz(None, 0, p, p, 128, 128, None) == 1
+    assert qz(p, 1, mis, p, 128, 128, None) == 2
