@@ -40,7 +40,7 @@ constexpr int kDefaultMaxSmem = 232448;    // 227 KB opt-in per block on sm_100
 constexpr int kMaxStages = 12;
 static_assert(kMaxStages <= DONE_RING, "the done ring must cover every operand stage");
 constexpr int kMinStages = 2;
-constexpr int kMaxSplit = 4;
+constexpr int kMaxSplit = 8; // CTAs per split-K cluster (portable cluster size)
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull; // 2 s per pipeline wait
 
 // ------------------------------------------------------------------ devices
@@ -281,6 +281,11 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
             if (g_forced_split && split != g_forced_split)
                 continue;
             if (c.pair && split > 1)
+                continue;
+            // 8-CTA clusters only on request: measured slower than 4 on the
+            // decode shape (the 8-way reduction and cluster placement cost
+            // more than the shorter K range saves)
+            if (split > 4 && g_forced_split != split)
                 continue;
             if (split > 1) {
                 // split-K only for dense calls too small to fill the SMs

@@ -187,10 +187,10 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
 
 /* Test hook: pin block_m / block_n, the split-K factor and the CTA-pair mode
  * for later calls (0, 0 restores automatic tile choice; split 0 = automatic,
- * 1 = no split, 2 or 4 = that many CTAs per tile, used only where split-K
+ * 1 = no split, 2, 4 or 8 = that many CTAs per tile, used only where split-K
  * applies; cta_pair 0 = automatic, 1 = one CTA per tile, 2 = CTA pairs).
  * Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is built, the
- * split is not 0, 1, 2 or 4, or cta_pair is not 0, 1 or 2. */
+ * split is not 0, 1, 2, 4 or 8, or cta_pair is not 0, 1 or 2. */
 int dg_force_config(int block_m, int block_n, int split, int cta_pair);
 
 #ifdef __cplusplus

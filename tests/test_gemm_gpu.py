@@ -117,11 +117,13 @@ def test_dense_grouped_promotion_partial_steps(mw, bn):
 
 
 @pytest.mark.parametrize("mw,bn,split", [(1, 16, 2), (1, 64, 4), (1, 128, 2), (1, 112, 4),
-                                         (2, 32, 2), (1, 96, 4)])
+                                         (2, 32, 2), (1, 96, 4), (1, 128, 8), (1, 32, 8)])
 def test_dense_split_k(mw, bn, split):
     """Split-K over a thread-block cluster: ragged M and N, K blocks not a
     multiple of the split, reduction through distributed shared memory."""
-    prob = inputs.make_dense(100 if mw == 1 else 300, 336, 128 * 11, seed=300 + bn + split)
+    # 11 K blocks (19 for 8 CTAs: at least two per CTA), not a multiple of the split
+    prob = inputs.make_dense(100 if mw == 1 else 300, 336, 128 * (11 if split <= 4 else 19),
+                             seed=300 + bn + split)
     ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
     fp8.force_config(128 * mw, bn, split)
     try:
@@ -460,3 +462,38 @@ def test_quantize_full_size_then_gemm():
     rows = np.arange(0, M, 97)
     ref = oracle.gemm_dense(q[rows], sa[:, rows].copy(), prob.b, prob.sb, len(rows), N, K)
     H.assert_close(H.bf16_bits_to_f64(d)[rows], ref, "quantised then GEMM")
+
+
+# --------------------------------------------------------------------- many experts
+
+
+def test_contiguous_many_experts():
+    """64 experts with counts from 0 to 300 (many empty or single-block
+    segments), every row compared."""
+    G = 64
+    counts = [int(c) for c in np.random.default_rng(64).integers(0, 301, G)]
+    counts[5] = 0
+    counts[6] = 1
+    prob = inputs.make_contiguous(G, 256, 256, seed=64, counts=counts)
+    ref = oracle.gemm_contiguous(prob.a, prob.sa, prob.b, prob.sb, prob.m_indices,
+                                 prob.num_groups, prob.M_sum, prob.N, prob.K)
+    d = H.run_contiguous(prob)
+    check_status()
+    valid = prob.m_indices.numpy() >= 0
+    H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], "contiguous 64 experts")
+    assert H.untouched(d)[~valid].all()
+
+
+def test_masked_many_groups():
+    """256 groups of up to 64 rows (the device enumerates the tiles of every
+    group from masked_m), rows past masked_m untouched."""
+    G = 256
+    mm = [int(c) for c in np.random.default_rng(256).integers(0, 65, G)]
+    prob = inputs.make_masked(G, 64, 128, 256, seed=256, masked_m=mm)
+    ref = oracle.gemm_masked(prob.a, prob.sa, prob.b, prob.sb, prob.masked_m, prob.G,
+                             prob.M_max, prob.N, prob.K)
+    d = H.run_masked(prob)
+    check_status()
+    valid = ~np.isnan(ref)
+    H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], "masked 256 groups")
+    assert H.untouched(d)[~valid].all()
