@@ -426,8 +426,24 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     // D as a [rows][N] BF16 matrix; the epilogue stores 32 x 32 boxes staged
     // with the 64-byte swizzle (elements past the tensor are not written)
     const long d_rows = pb.kind == DG_KIND_MASKED ? (long)groups * pb.M : pb.M;
-    if ((st = make_tmap_2d(&tmap_d, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pb.N, d_rows, pb.N, 32,
-                           32, CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
+    // When N and every epilogue thread's column span are multiples of 32,
+    // D is viewed in 3-D as [N/32 column chunks][rows][32 columns] so that a
+    // warp's whole staged row block (chunk-major, as staged) is one box.
+    const int thread_cols = cand->mw == 1 ? cfg.block_n / 2 : cfg.block_n;
+    bool d3 = cfg.split == 1 && pb.N % 32 == 0 && thread_cols % 32 == 0;
+    if (d3) {
+        EncodeTiledFn fn = encode_fn();
+        cuuint64_t dims[3] = {32, (cuuint64_t)d_rows, (cuuint64_t)(pb.N / 32)};
+        cuuint64_t strides[2] = {(cuuint64_t)pb.N * 2, 64};
+        cuuint32_t box[3] = {32, 32, (cuuint32_t)(thread_cols / 32)};
+        cuuint32_t estr[3] = {1, 1, 1};
+        d3 = fn && fn(&tmap_d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, D, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    if (!d3 && (st = make_tmap_2d(&tmap_d, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pb.N, d_rows,
+                                  pb.N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != DG_OK)
         return st;
 
     Params p;
@@ -452,6 +468,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     p.m_indices = m_indices;
     p.masked_m = masked_m;
     p.D = static_cast<uint16_t *>(D);
+    p.d_store_3d = d3 ? 1 : 0;
     p.status = dev->status;
     p.timeout_ns = wait_timeout_ns();
 

@@ -907,6 +907,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             fence_proxy_async_smem();
             __syncwarp();
             bool issued = false;
+            if (use_tma && p.d_store_3d) {
+                // every chunk is full: the warp's whole row block is one 3-D
+                // box ([chunk][row][32 columns], the staging layout)
+                if (lane == 0)
+                    tma_store_3d(&tmap_d, stg_w, 0, warp_row0, cbase >> 5);
+                issued = true;
+            } else {
 #pragma unroll
             for (int c = 0; c < NC; c += 32) {
                 const uint32_t stg = stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES;
@@ -929,6 +936,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
+            } // 2-D chunks
             if (issued && lane == 0)
                 bulk_commit_group();
         }

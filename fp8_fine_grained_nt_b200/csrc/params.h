@@ -70,6 +70,7 @@ struct Params {
     const int *m_indices;
     const int *masked_m;
     uint16_t *D;    // BF16 bits
+    int d_store_3d; // 1: tmap_d is the 3-D [N/32][rows][32] view (one TMA store per warp)
     unsigned int *status; // device status word (DEVERR_* bits)
     uint64_t timeout_ns;  // limit on any single pipeline wait
 };
