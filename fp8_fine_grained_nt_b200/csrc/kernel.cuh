@@ -9,19 +9,26 @@
 // and BF16 output.
 //
 // Roles (384 threads, one CTA per SM, persistent over output tiles):
-//   warp 0      TMA producer: A / B tiles into a multi-stage shared-memory
-//               ring (the A and B copies of a stage issued by two lanes in one
-//               instruction), the tile's RHS scales into a per-tile slot
-//               (cp.async).  The README's data-movement warpgroup, reduced to
-//               one warp.
+//   warp 0      TMA producer of the A tiles (one lane per 128-row half).
+//   warp 2      TMA producer of the B tiles; at set-up it also counts the
+//               masked form's tiles per group.  The two producers' copies of a
+//               stage meet on one full barrier (two arrivals, each with its
+//               byte count), so their issue latencies overlap.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer: one
 //               128-K block per MMA group into a ring of TMEM buffers, fresh
-//               accumulation per block so each block's partial stays separable.
+//               accumulation per block so each block's partial stays
+//               separable; one commit per K block frees the operand stage and
+//               publishes the partial.
+//   warp 3      scale producer: the tile's RHS scales (cp.async) and the LHS
+//               scales of the CTA's rows, several K blocks per TMA box, into
+//               two small rings the epilogue releases.
 //   warps 4-11  promotion epilogue: tcgen05.ld of the blocks' partials, FMA
-//               with sa*sb into FP32 registers (sa read from global memory a
-//               few blocks ahead), BF16 conversion and a coalesced store at
-//               tile end.
-// Warps 2-3 only help with set-up (masked tile counts).
+//               with sa*sb into FP32 registers, then BF16 into a shared
+//               staging tile and asynchronous TMA stores.
+// Variants: PAIR (a cluster of two CTAs computes a 256-row tile with
+// cta_group::2 MMAs), SCALAR (per-tensor scaling: the whole K range
+// accumulates in TMEM and the epilogue reads each tile once), and split-K
+// over a thread-block cluster (runtime, dense only).
 //
 // Tile shape: BLOCK_M = 128 * MW rows (MW = 2 issues two M=128 MMAs that share
 // the B tile), BLOCK_N = BN columns, BN a multiple of 16 in [16, 256] so that
