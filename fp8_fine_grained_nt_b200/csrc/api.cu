@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <math.h>
 #include <mutex>
 #include <stdint.h>
@@ -62,9 +63,27 @@ struct DeviceInfo {
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
-int g_num_sms_limit = 0;
-int g_forced_bm = 0, g_forced_bn = 0, g_forced_split = 0, g_forced_pair = 0;
-uint64_t g_timeout_ns = 0;
+// Settings shared by every call (a caller may set them from any thread):
+// the SM bound of set_num_sms and the test hook of dg_force_config, the
+// latter packed into one word so that a call sees one consistent setting.
+std::atomic<int> g_num_sms_limit{0};
+std::atomic<uint32_t> g_forced{0};
+
+struct Forced {
+    int bm, bn, split, pair;
+};
+
+uint32_t pack_forced(int bm, int bn, int split, int pair)
+{
+    return (uint32_t)bm | ((uint32_t)bn << 10) | ((uint32_t)split << 20) | ((uint32_t)pair << 24);
+}
+
+Forced forced_config()
+{
+    const uint32_t w = g_forced.load(std::memory_order_relaxed);
+    return Forced{(int)(w & 0x3FF), (int)((w >> 10) & 0x3FF), (int)((w >> 20) & 0xF),
+                  (int)((w >> 24) & 0x3)};
+}
 
 int device_info(DeviceInfo **out)
 {
@@ -94,12 +113,13 @@ int device_info(DeviceInfo **out)
 
 uint64_t wait_timeout_ns()
 {
-    if (g_timeout_ns == 0) {
+    // read once (thread-safe static initialisation)
+    static const uint64_t timeout_ns = [] {
         const char *env = getenv("DG_WAIT_TIMEOUT_MS");
-        long ms = env ? atol(env) : 0;
-        g_timeout_ns = ms > 0 ? (uint64_t)ms * 1000000ull : kDefaultTimeoutNs;
-    }
-    return g_timeout_ns;
+        const long ms = env ? atol(env) : 0;
+        return ms > 0 ? (uint64_t)ms * 1000000ull : kDefaultTimeoutNs;
+    }();
+    return timeout_ns;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -258,6 +278,7 @@ int max_resident_clusters(int split, int sms)
 int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand, dg_config *cfg,
            SmemPlan *plan)
 {
+    const Forced forced = forced_config();
     const Candidate *best = nullptr;
     int best_split = 1;
     double best_cost = 0;
@@ -265,27 +286,27 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     for (int i = 0; i < kNumCandidates; ++i) {
         const Candidate &c = kCandidates[i];
         const int c_bm = c.pair ? 256 : c.mw * 128;
-        if (g_forced_bm && (c_bm != g_forced_bm || c.bn != g_forced_bn))
+        if (forced.bm && (c_bm != forced.bm || c.bn != forced.bn))
             continue;
-        if (g_forced_pair && (g_forced_pair == 2) != (c.pair != 0))
+        if (forced.pair && (forced.pair == 2) != (c.pair != 0))
             continue;
         // CTA pairs only on request: measured on B200 they were no faster
         // than one CTA per tile on the dense, masked and 256-row shapes
-        if (c.pair && g_forced_pair != 2)
+        if (c.pair && forced.pair != 2)
             continue;
         if (pb.kind == DG_KIND_CONTIGUOUS && c_bm != 128)
             continue; // a 256-row tile could straddle two 128-aligned experts
         if ((pb.kind == DG_KIND_DENSE_PER_TENSOR) != (c.scalar != 0))
             continue; // per-tensor and fine-grained scaling have their own kernels
         for (int split = 1; split <= kMaxSplit; split *= 2) {
-            if (g_forced_split && split != g_forced_split)
+            if (forced.split && split != forced.split)
                 continue;
             if (c.pair && split > 1)
                 continue;
             // 8-CTA clusters only on request: measured slower than 4 on the
             // decode shape (the 8-way reduction and cluster placement cost
             // more than the shorter K range saves)
-            if (split > 4 && g_forced_split != split)
+            if (split > 4 && forced.split != split)
                 continue;
             if (split > 1) {
                 // split-K only for dense calls too small to fill the SMs
@@ -356,8 +377,9 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
 int effective_sms(const DeviceInfo *d)
 {
     int n = d ? d->sm_count : kDefaultSms;
-    if (g_num_sms_limit > 0 && g_num_sms_limit < n)
-        n = g_num_sms_limit;
+    const int limit = g_num_sms_limit.load(std::memory_order_relaxed);
+    if (limit > 0 && limit < n)
+        n = limit;
     return n;
 }
 
@@ -592,7 +614,7 @@ int get_tma_aligned_size(int x, int element_size)
 
 int set_num_sms(int n)
 {
-    g_num_sms_limit = n > 0 ? n : 0;
+    g_num_sms_limit.store(n > 0 ? n : 0, std::memory_order_relaxed);
     return DG_OK;
 }
 
@@ -602,12 +624,13 @@ int get_num_sms(void)
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
-        if (g_num_sms_limit > 0 && g_num_sms_limit < count)
-            return g_num_sms_limit;
+        const int limit = g_num_sms_limit.load(std::memory_order_relaxed);
+        if (limit > 0 && limit < count)
+            return limit;
         return count;
     }
     cudaGetLastError(); // no device: clear the sticky-free error state
-    return g_num_sms_limit;
+    return g_num_sms_limit.load(std::memory_order_relaxed);
 }
 
 const char *dg_status_string(int status)
@@ -657,7 +680,8 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
         return DG_ERR_UNSUPPORTED_SHAPE;
     if (kind == DG_KIND_MASKED && num_groups > MAX_MASKED_GROUPS)
         return DG_ERR_UNSUPPORTED_SHAPE;
-    int sms = num_sms > 0 ? num_sms : (g_num_sms_limit > 0 ? g_num_sms_limit : kDefaultSms);
+    const int limit = g_num_sms_limit.load(std::memory_order_relaxed);
+    int sms = num_sms > 0 ? num_sms : (limit > 0 ? limit : kDefaultSms);
     const bool one_group = kind == DG_KIND_DENSE || kind == DG_KIND_DENSE_PER_TENSOR;
     Problem pb{kind, M, N, K, one_group ? 1 : num_groups, expected_m};
     const Candidate *cand = nullptr;
@@ -672,19 +696,14 @@ int dg_force_config(int block_m, int block_n, int split, int cta_pair)
     if (cta_pair < 0 || cta_pair > 2)
         return DG_ERR_UNSUPPORTED_SHAPE;
     if (block_m == 0 && block_n == 0) {
-        g_forced_bm = g_forced_bn = 0;
-        g_forced_split = split;
-        g_forced_pair = cta_pair;
+        g_forced.store(pack_forced(0, 0, split, cta_pair), std::memory_order_relaxed);
         return DG_OK;
     }
     for (int i = 0; i < kNumCandidates; ++i) {
         const Candidate &c = kCandidates[i];
         if ((c.pair ? 256 : c.mw * 128) == block_m && c.bn == block_n &&
             (cta_pair == 0 || (cta_pair == 2) == (c.pair != 0))) {
-            g_forced_bm = block_m;
-            g_forced_bn = block_n;
-            g_forced_split = split;
-            g_forced_pair = cta_pair;
+            g_forced.store(pack_forced(block_m, block_n, split, cta_pair), std::memory_order_relaxed);
             return DG_OK;
         }
     }

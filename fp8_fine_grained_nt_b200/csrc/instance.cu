@@ -3,6 +3,8 @@
 // -DFP8NT_MW, -DFP8NT_BN, -DFP8NT_PAIR and -DFP8NT_SCALAR.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "kernel.cuh"
 #include "launch.h"
 
@@ -27,20 +29,30 @@ namespace fp8nt {
 cudaError_t FP8NT_NAME(FP8NT_MW, FP8NT_BN, FP8NT_PAIR, FP8NT_SCALAR)(const LaunchArgs &args)
 {
     auto kernel = fp8_gemm_kernel<FP8NT_MW, FP8NT_BN, FP8NT_PAIR != 0, FP8NT_SCALAR != 0>;
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           args.smem_bytes);
-    if (err != cudaSuccess)
-        return err;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    // The dynamic shared-memory limit is raised once per device to the
+    // largest size requested so far (a per-call attribute update costs host
+    // time on every launch).
+    static std::atomic<int> smem_limit[64];
+    if (smem_limit[dev].load(std::memory_order_acquire) < args.smem_bytes) {
+        cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               args.smem_bytes);
+        if (err != cudaSuccess)
+            return err;
+        int seen = smem_limit[dev].load(std::memory_order_relaxed);
+        while (seen < args.smem_bytes &&
+               !smem_limit[dev].compare_exchange_weak(seen, args.smem_bytes)) {
+        }
+    }
     cudaLaunchConfig_t cfg = {};
     int grid = args.grid;
     if (FP8NT_PAIR && args.cluster == 2) {
         // persistent pairs: no more than can be resident at once (a GPC with
         // an odd number of free SMs holds one CTA fewer than a naive count)
-        static int max_pairs[64] = {};
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-            return cudaErrorInvalidDevice;
-        if (max_pairs[dev] == 0) {
+        static std::atomic<int> max_pairs[64];
+        if (max_pairs[dev].load(std::memory_order_relaxed) == 0) {
             cudaLaunchConfig_t q = {};
             q.gridDim = dim3((unsigned)args.grid, 1, 1);
             q.blockDim = dim3(NUM_THREADS, 1, 1);
