@@ -340,9 +340,10 @@ def run_reference(args):
 def measure_next_rows(fp8, peaks, iters: int = 20) -> dict:
     """The rows built beyond the fine-grained GEMM, each timed alone (CUDA
     events around every call, L2 flushed before each): the 1x128 activation
-    quantiser and the per-tensor-scale GEMM."""
+    quantiser, the per-tensor-scale GEMM and a skewed (Zipf-like) expert load
+    for the contiguous grouped GEMM."""
     dev = "cuda"
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def timed(fn) -> float:
@@ -350,7 +351,7 @@ def measure_next_rows(fp8, peaks, iters: int = 20) -> dict:
             fn()
         total = 0.0
         for _ in range(iters):
-            flush.zero_()
+            flush.max()  # reads 256 MB: evicts L2 without leaving dirty lines
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -385,6 +386,20 @@ def measure_next_rows(fp8, peaks, iters: int = 20) -> dict:
     out[f"per_tensor_gemm_{M}x{N}x{K}"] = {
         "us": round(t * 1e6, 2), "tflops": round(flop / t / 1e12, 1), "flop": flop,
         "bound": "tensor", "roofline_frac": round(flop / t / 1e12 / peak, 4)}
+    # skewed expert load: counts ~ Zipf(1.2) over 8 experts, 32768 tokens in
+    # all, each segment padded to the alignment (the contiguous workload's N, K)
+    from fp8_fine_grained_nt_b200 import inputs
+    weights = np.array([1.0 / (e + 1) ** 1.2 for e in range(8)])
+    counts = [int(round(c)) for c in 32768 * weights / weights.sum()]
+    prob = inputs.make_contiguous(8, 4096, 7168, seed=7, counts=counts)
+    a, sa_c, b, sb_c = (prob.a.to(dev), prob.sa.to(dev), prob.b.to(dev), prob.sb.to(dev))
+    mi = prob.m_indices.to(dev)
+    d = torch.empty(prob.M_sum, 4096, dtype=torch.bfloat16, device=dev)
+    t = timed(lambda: fp8.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(a, sa_c, b, sb_c, d, mi))
+    flop = 2 * sum(counts) * 4096 * 7168
+    out["contiguous_zipf_8x4096x7168"] = {
+        "us": round(t * 1e6, 2), "tflops": round(flop / t / 1e12, 1), "flop": flop,
+        "counts": counts, "bound": "tensor", "roofline_frac": round(flop / t / 1e12 / peak, 4)}
     status = fp8.get_device_status()
     if status != 0:
         raise RuntimeError(f"device status after the extra rows: {fp8.status_string(status)}")

@@ -498,3 +498,17 @@ def test_masked_many_groups():
     valid = ~np.isnan(ref)
     H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], "masked 256 groups")
     assert H.untouched(d)[~valid].all()
+
+
+def test_contiguous_skewed_experts():
+    """A Zipf-like expert load (most tokens on a few experts, some experts
+    empty), every row compared."""
+    counts = [1500, 700, 260, 90, 31, 7, 1, 0]
+    prob = inputs.make_contiguous(8, 384, 512, seed=99, counts=counts)
+    ref = oracle.gemm_contiguous(prob.a, prob.sa, prob.b, prob.sb, prob.m_indices,
+                                 prob.num_groups, prob.M_sum, prob.N, prob.K)
+    d = H.run_contiguous(prob)
+    check_status()
+    valid = prob.m_indices.numpy() >= 0
+    H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], "contiguous skewed")
+    assert H.untouched(d)[~valid].all()
