@@ -31,6 +31,7 @@ __all__ = [
     "set_num_sms",
     "get_num_sms",
     "get_device_status",
+    "selftest_wait_timeout",
     "select_config",
     "force_config",
     "status_string",
@@ -84,6 +85,7 @@ def load_library():
         lib.gemm_fp8_fp8_bf16_nt.argtypes = [P, P, P, P, P, I, I, I, P]
         lib.gemm_fp8_fp8_bf16_nt_per_tensor.argtypes = [P, P, P, P, P, I, I, I, P]
         lib.quantize_fp8_1x128.argtypes = [P, I, P, P, I, I, P]
+        lib.dg_selftest_wait_timeout.argtypes = [I, P]
         lib.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         lib.m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.get_m_alignment_for_contiguous_layout.argtypes = []
@@ -263,6 +265,14 @@ def set_num_sms(n: int) -> None:
 
 def get_num_sms() -> int:
     return load_library().get_num_sms()
+
+
+def selftest_wait_timeout(timeout_us: int = 20000, stream=None) -> None:
+    """Enqueue the bounded-wait self-test: a device wait that nothing satisfies
+    gives up after timeout_us and records DG_ERR_DEVICE_TIMEOUT (read it with
+    get_device_status())."""
+    _check(load_library().dg_selftest_wait_timeout(int(timeout_us), _stream_ptr(stream)),
+           "dg_selftest_wait_timeout")
 
 
 def get_device_status(stream=None) -> int:

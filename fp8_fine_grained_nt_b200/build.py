@@ -120,7 +120,9 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -
     jobs = jobs or max(1, os.cpu_count() or 1)
     tasks = [(os.path.join(CSRC, "api.cu"), os.path.join(BUILD_DIR, "api.o"), [], "api"),
              (os.path.join(CSRC, "quantize.cu"), os.path.join(BUILD_DIR, "quantize.o"), [],
-              "quantize")]
+              "quantize"),
+             (os.path.join(CSRC, "selftest.cu"), os.path.join(BUILD_DIR, "selftest.o"), [],
+              "selftest")]
     for mw, bn, pair, scalar in kernel_list():
         tag = f"mw{mw}_bn{bn}_p{pair}_s{scalar}"
         tasks.append((os.path.join(CSRC, "instance.cu"), os.path.join(BUILD_DIR, f"kernel_{tag}.o"),

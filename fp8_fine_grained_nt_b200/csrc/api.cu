@@ -602,6 +602,20 @@ int quantize_fp8_1x128(const void *x, int x_dtype, void *q, float *sa, int M, in
                : DG_ERR_CUDA;
 }
 
+int dg_selftest_wait_timeout(int timeout_us, dg_stream_t stream)
+{
+    if (timeout_us <= 0 || timeout_us > 10000000)
+        return DG_ERR_INVALID_ARGUMENT;
+    DeviceInfo *dev = nullptr;
+    int st = device_info(&dev);
+    if (st != DG_OK)
+        return st;
+    return launch_wait_timeout_selftest(dev->status, (unsigned long long)timeout_us * 1000ull,
+                                        reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DG_OK
+               : DG_ERR_CUDA;
+}
+
 int get_m_alignment_for_contiguous_layout(void) { return 128; }
 
 int get_tma_aligned_size(int x, int element_size)

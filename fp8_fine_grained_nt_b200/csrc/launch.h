@@ -23,6 +23,10 @@ struct LaunchArgs {
 
 typedef cudaError_t (*LaunchFn)(const LaunchArgs &);
 
+// Bounded-wait self-test (csrc/selftest.cu).
+cudaError_t launch_wait_timeout_selftest(unsigned int *status, unsigned long long timeout_ns,
+                                         cudaStream_t stream);
+
 // 1x128 activation quantiser (csrc/quantize.cu).
 cudaError_t launch_quantize_1x128(const void *x, bool bf16_in, uint8_t *q, float *sa, int M, int K,
                                   long ld_sa, cudaStream_t stream);

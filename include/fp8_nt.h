@@ -148,6 +148,14 @@ int get_tma_aligned_size(int x, int element_size);
 int set_num_sms(int n);
 int get_num_sms(void);
 
+/* Self-test of the device-side error path (no counterpart in the pages): one
+ * thread waits, with the bounded mbarrier wait every pipeline role uses, on a
+ * barrier nothing arrives on.  After timeout_us microseconds (1..10^7) the
+ * wait gives up and records DG_ERR_DEVICE_TIMEOUT in the device status word,
+ * which dg_get_device_status() then returns; the kernel ends by itself and
+ * the context stays usable.  Returns DG_OK once the kernel is enqueued. */
+int dg_selftest_wait_timeout(int timeout_us, dg_stream_t stream);
+
 /* Static description of a dg_status value. */
 const char *dg_status_string(int status);
 

@@ -512,3 +512,20 @@ def test_contiguous_skewed_experts():
     valid = prob.m_indices.numpy() >= 0
     H.assert_close(H.bf16_bits_to_f64(d)[valid], ref[valid], "contiguous skewed")
     assert H.untouched(d)[~valid].all()
+
+
+# --------------------------------------------------------------------- failure detection
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A device wait that nothing satisfies gives up after its limit and is
+    reported through the status word; no fault, and later calls still work."""
+    assert fp8.get_device_status() == 0
+    fp8.selftest_wait_timeout(20000)  # 20 ms
+    assert fp8.get_device_status() == 6, "expected DG_ERR_DEVICE_TIMEOUT"
+    assert fp8.get_device_status() == 0, "status word not cleared"
+    prob = inputs.make_dense(130, 200, 384, seed=8)
+    ref = oracle.gemm_dense(prob.a, prob.sa, prob.b, prob.sb, prob.M, prob.N, prob.K)
+    d = H.run_dense(prob)
+    check_status()
+    H.assert_close(H.bf16_bits_to_f64(d), ref, "after the timeout self-test")

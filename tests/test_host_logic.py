@@ -255,3 +255,9 @@ def test_quantize_host_checks(lib):
     assert qz(p, 0, p, p, 0, 128, None) == 0     # empty
     assert qz(None, 0, p, p, 128, 128, None) == 1
     assert qz(p, 1, mis, p, 128, 128, None) == 2
+
+
+def test_selftest_rejects_bad_timeouts(lib):
+    assert lib.dg_selftest_wait_timeout(0, None) == 1
+    assert lib.dg_selftest_wait_timeout(-5, None) == 1
+    assert lib.dg_selftest_wait_timeout(20000001, None) == 1
