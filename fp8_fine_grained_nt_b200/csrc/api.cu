@@ -253,12 +253,26 @@ int plan_for(const Problem &pb, int mw, int bn, int split, int pair, int max_sme
 {
     const int nkb = pb.K / 128;
     const int prefix_ints = pb.kind == DG_KIND_MASKED ? 2 * pb.groups + 1 : 0;
-    for (int s = kMaxStages; s >= kMinStages; --s) {
-        SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints, split > 1, pair != 0);
-        if ((int)p.total + 1024 <= max_smem) {
-            *stages = s;
-            *plan = p;
-            return DG_OK;
+    // Shared memory beyond the operand ring holds the output staging: the
+    // whole BF16 tile (one bulk store per warp), or fewer 2 KB slots that
+    // the output chunks stream through.  With per-block promotion the
+    // epilogue bounds the kernel and a whole staged tile is faster than an
+    // extra operand stage; with per-tensor scales the operand ring bounds it
+    // and the extra stage wins (measured on B200: 4096x7168x2048 per-tensor
+    // 60 -> 54 us with 4 stages and one slot; fine-grained 79 -> 84 us).
+    const int chunks = ((mw == 1 ? bn / 2 : bn) + 31) / 32;
+    const bool stages_first = pb.kind == DG_KIND_DENSE_PER_TENSOR;
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int s = kMaxStages; s >= kMinStages; --s) {
+            const int lo = (stages_first || pass == 1) ? 1 : chunks;
+            for (int slots = chunks; slots >= lo; --slots) {
+                SmemPlan p = make_smem_plan(mw, bn, s, nkb, prefix_ints, split > 1, pair != 0, slots);
+                if ((int)p.total + 1024 <= max_smem) {
+                    *stages = s;
+                    *plan = p;
+                    return DG_OK;
+                }
+            }
         }
     }
     return DG_ERR_UNSUPPORTED_SHAPE;
@@ -452,7 +466,8 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     // D is viewed in 3-D as [N/32 column chunks][rows][32 columns] so that a
     // warp's whole staged row block (chunk-major, as staged) is one box.
     const int thread_cols = cand->mw == 1 ? cfg.block_n / 2 : cfg.block_n;
-    bool d3 = cfg.split == 1 && pb.N % 32 == 0 && thread_cols % 32 == 0;
+    bool d3 = cfg.split == 1 && pb.N % 32 == 0 && thread_cols % 32 == 0 &&
+              (int)plan.out_slots * 32 >= thread_cols; // whole row block staged
     if (d3) {
         EncodeTiledFn fn = encode_fn();
         cuuint64_t dims[3] = {32, (cuuint64_t)d_rows, (cuuint64_t)(pb.N / 32)};

@@ -890,18 +890,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // stores of whole 64-byte row segments.
             const uint32_t row_mask = __ballot_sync(0xffffffffu, row_ok);
             const bool use_tma = row_mask != 0u && (row_mask == 0xffffffffu || p.kind == KIND_DENSE);
+            const int slots = (int)plan.out_slots; // 2 KB chunk slots of this warp
             const uint32_t stg_w = smem_addr(smem + plan.off_out) +
-                                   (uint32_t)ew * (uint32_t)(T::OUT_CHUNKS * OUT_STAGE_BYTES);
+                                   (uint32_t)ew * (uint32_t)(slots * OUT_STAGE_BYTES);
             const int warp_row0 = ti.d_row0 + half * HALF_M + q * 32;
             const int rd_sub = lane >> 2;  // row within an 8-row group (read side)
             const int rd_piece = lane & 3; // 16-byte piece within a 64-byte row chunk
-            // the previous tile's TMA stores must have read this warp's buffer
-            if (lane == 0)
-                bulk_wait_read_all();
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < NC; c += 32) {
-                const uint32_t stg = stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES;
+            auto stage_chunk = [&](int c, uint32_t stg) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (c + 8 * j < NC)
@@ -910,42 +905,79 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                      pack_bf16x2(acc[c + 8 * j + 2], acc[c + 8 * j + 3]),
                                      pack_bf16x2(acc[c + 8 * j + 4], acc[c + 8 * j + 5]),
                                      pack_bf16x2(acc[c + 8 * j + 6], acc[c + 8 * j + 7]));
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            bool issued = false;
-            if (use_tma && p.d_store_3d) {
-                // every chunk is full: the warp's whole row block is one 3-D
-                // box ([chunk][row][32 columns], the staging layout)
+            };
+            auto store_chunk_plain = [&](int c, uint32_t stg) {
+                const int col = cbase + c + 8 * rd_piece;
+                const bool col_ok = (c + 8 * rd_piece < NC) && col < p.N;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = i * 8 + rd_sub;
+                    if (col_ok && ((row_mask >> r) & 1u)) {
+                        const uint4 v = ld_shared_v4(stg + r * 64 + ((rd_piece ^ ((r >> 1) & 3)) << 4));
+                        st_global_v4(p.D + (size_t)(warp_row0 + r) * p.N + col, v.x, v.y, v.z, v.w);
+                    }
+                }
+            };
+            if (slots >= T::OUT_CHUNKS) {
+                // the whole row block is staged: the previous tile's TMA
+                // stores must have read the buffer
                 if (lane == 0)
-                    tma_store_3d(&tmap_d, stg_w, 0, warp_row0, cbase >> 5);
-                issued = true;
-            } else {
+                    bulk_wait_read_all();
+                __syncwarp();
 #pragma unroll
-            for (int c = 0; c < NC; c += 32) {
-                const uint32_t stg = stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES;
-                if (use_tma && c + 32 <= NC) {
+                for (int c = 0; c < NC; c += 32)
+                    stage_chunk(c, stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES);
+                fence_proxy_async_smem();
+                __syncwarp();
+                bool issued = false;
+                if (use_tma && p.d_store_3d) {
+                    // every chunk is full: one 3-D box ([chunk][row][32 columns],
+                    // the staging layout)
                     if (lane == 0)
-                        tma_store_2d(&tmap_d, stg, cbase + c, warp_row0);
+                        tma_store_3d(&tmap_d, stg_w, 0, warp_row0, cbase >> 5);
                     issued = true;
-                } else if (row_mask != 0u) {
-                    const int col = cbase + c + 8 * rd_piece;
-                    const bool col_ok = (c + 8 * rd_piece < NC) && col < p.N;
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = i * 8 + rd_sub;
-                        if (col_ok && ((row_mask >> r) & 1u)) {
-                            const uint4 v =
-                                ld_shared_v4(stg + r * 64 + ((rd_piece ^ ((r >> 1) & 3)) << 4));
-                            st_global_v4(p.D + (size_t)(warp_row0 + r) * p.N + col, v.x, v.y, v.z,
-                                         v.w);
+                    for (int c = 0; c < NC; c += 32) {
+                        const uint32_t stg = stg_w + (uint32_t)(c / 32) * OUT_STAGE_BYTES;
+                        if (use_tma && c + 32 <= NC) {
+                            if (lane == 0)
+                                tma_store_2d(&tmap_d, stg, cbase + c, warp_row0);
+                            issued = true;
+                        } else if (row_mask != 0u) {
+                            store_chunk_plain(c, stg);
                         }
                     }
                 }
+                if (issued && lane == 0)
+                    bulk_commit_group();
+            } else {
+                // fewer slots than chunks: the chunks stream through the
+                // slots, a slot being rewritten only after the TMA store that
+                // read it has finished reading (so more operand stages fit)
+#pragma unroll
+                for (int c = 0; c < NC; c += 32) {
+                    const int k = c / 32;
+                    const uint32_t stg = stg_w + (uint32_t)(k % slots) * OUT_STAGE_BYTES;
+                    if (k % slots == 0) {
+                        if (lane == 0)
+                            bulk_wait_read_all();
+                        __syncwarp();
+                    }
+                    stage_chunk(c, stg);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (use_tma && c + 32 <= NC) {
+                        if (lane == 0) {
+                            tma_store_2d(&tmap_d, stg, cbase + c, warp_row0);
+                            bulk_commit_group();
+                        }
+                    } else if (row_mask != 0u) {
+                        store_chunk_plain(c, stg);
+                    }
+                    __syncwarp(); // the plain path's reads finish before the slot is reused
+                }
             }
-            } // 2-D chunks
-            if (issued && lane == 0)
-                bulk_commit_group();
         }
         // every TMA store has completed before the CTA exits
         if (lane == 0)

@@ -41,7 +41,8 @@ struct SmemPlan {
     uint32_t off_sb;        // RHS-scale tile slots: 2 x 3 x sb_pitch floats
     uint32_t sb_pitch;      // floats per sb row in smem (nkb rounded up to 4)
     uint32_t off_sa;        // LHS-scale ring: 2 x SA_SLOT_BYTES
-    uint32_t off_out;       // output staging: the whole BF16 tile, 2 KB chunks per epilogue warp
+    uint32_t off_out;       // output staging: out_slots 2 KB chunk slots per epilogue warp
+    uint32_t out_slots;     // = the warp's chunk count (whole tile staged) or fewer (streamed)
     uint32_t off_red;       // split-K: this CTA's FP32 partial tile, rows padded by RED_PAD
     uint32_t off_prefix;    // masked: (G + 1) ints of per-group tile prefix sums
     uint32_t off_bars;      // all mbarriers
@@ -83,7 +84,8 @@ __host__ __device__ inline uint32_t align_up_u32(uint32_t x, uint32_t a)
 // Shared-memory layout for a (MW, BN) kernel with the given ring depths; a
 // CTA of a pair holds half of the B tile.
 __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, int nkb,
-                                                   int prefix_ints, bool split_k, bool pair = false)
+                                                   int prefix_ints, bool split_k, bool pair = false,
+                                                   int out_slots = 0)
 {
     SmemPlan p;
     p.a_bytes = (uint32_t)mw * HALF_M * BLOCK_K;
@@ -97,9 +99,10 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     off = p.off_sa + 2u * SA_SLOT_BYTES;
     p.off_out = align_up_u32(off, 1024);
     // (split-K CTAs reduce through distributed shared memory and store
-    // directly: no output staging)
+    // directly: no output staging; out_slots <= 0 stages every chunk)
     const uint32_t out_chunks = split_k ? 0u : (uint32_t)((mw == 1 ? bn / 2 : bn) + 31) / 32;
-    off = p.off_out + NUM_EPI_WARPS * out_chunks * OUT_STAGE_BYTES;
+    p.out_slots = (out_slots > 0 && (uint32_t)out_slots < out_chunks) ? (uint32_t)out_slots : out_chunks;
+    off = p.off_out + NUM_EPI_WARPS * p.out_slots * OUT_STAGE_BYTES;
     p.off_red = align_up_u32(off, 128);
     if (split_k)
         off = p.off_red + (uint32_t)mw * HALF_M * (uint32_t)(bn + RED_PAD) * 4u;
