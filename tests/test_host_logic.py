@@ -261,3 +261,21 @@ def test_selftest_rejects_bad_timeouts(lib):
     assert lib.dg_selftest_wait_timeout(0, None) == 1
     assert lib.dg_selftest_wait_timeout(-5, None) == 1
     assert lib.dg_selftest_wait_timeout(20000001, None) == 1
+
+
+def test_shared_memory_plan_policy(lib):
+    """The per-tensor kernel, bound by its operand ring, trades the staged
+    output tile for an extra operand stage; the fine-grained kernels, bound by
+    the promotion epilogue, keep the whole staged tile.  Both fit the 227 KB
+    opt-in limit of a B200 block."""
+    limit = 232448
+    pt = fp8.select_config(fp8.KIND_DENSE_PER_TENSOR, 4096, 7168, 2048, num_sms=148)
+    fg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
+    assert pt["block_n"] == fg["block_n"] == 256 and pt["block_m"] == fg["block_m"] == 128
+    assert pt["stages"] == fg["stages"] + 1
+    # a whole 128x256 BF16 tile is 64 KB of staging; one 2 KB slot per warp is 16 KB
+    stage = 128 * 128 + 256 * 128
+    assert fg["smem_bytes"] - (fg["stages"] * stage) >= 64 * 1024
+    assert pt["smem_bytes"] - (pt["stages"] * stage) < 64 * 1024
+    for cfg in (pt, fg):
+        assert cfg["smem_bytes"] <= limit
