@@ -2,18 +2,21 @@
 
 One step = one call of each measured workload through the library's C ABI,
 inputs resident in HBM:
-  dense decode 64x2112x7168, dense prefill 4096x7168x2048 and 256x7168x2048,
-  contiguous m-grouped 8 experts x (4096, 7168), masked m-grouped 16 x 256 for
-  (N, K) = (4096, 7168) and (7168, 2048).
+  dense 128x128x512, dense decode 64x2112x7168, dense prefill 4096x7168x2048
+  and 256x7168x2048, contiguous m-grouped 8 experts x (4096, 7168), masked
+  m-grouped 16 x 256 for (N, K) = (4096, 7168) and (7168, 2048).
 Inputs are the seeded synthetic workloads of fp8_fine_grained_nt_b200.inputs.
 `value` = total algorithmic FLOP of a step / device time of a step (CUDA events,
 max over ranks).  `e2e` times the same step through the same C-ABI calls with
 the inputs in pinned host memory: host-to-device copies, the GEMMs and the
 device-to-host copy of every output inside the timed region.
 
-Multi-GPU (torchrun): every rank runs its own full step on its own GPU
-(independent problems, no collective on the data path); value = all ranks'
-FLOP / max-over-ranks time, "scaling": "weak".
+Multi-GPU: `--gpus N` runs N ranks, one per GPU (under torchrun, or spawned
+by this script through torch.distributed.run when WORLD_SIZE is unset).  Each
+rank computes its own shard of every workload, with no exchange between ranks
+(shard_problem: dense calls split N into 128-column blocks, the contiguous
+form splits experts, the masked form splits groups); value = FLOP of the whole
+workloads / max-over-ranks time, "scaling": "strong".
 
 --impl reference times the CPU oracle (the only reference that exists for this
 path) on a bounded sample of the same workloads, on rank 0 only.
@@ -46,6 +49,7 @@ NOMINAL_FP8_TFLOPS = 4500.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 WORKLOAD_NAMES = [
+    "dense_128x128x512",
     "dense_decode_64x2112x7168",
     "dense_prefill_4096x7168x2048",
     "dense_prefill_256x7168x2048",
@@ -53,9 +57,11 @@ WORKLOAD_NAMES = [
     "masked_16x256_4096x7168",
     "masked_16x256_7168x2048",
 ]
-WORKLOAD_DESC = ("decode 64x2112x7168 + prefill 4096x7168x2048 + prefill 256x7168x2048 + "
-                 "contiguous 8 experts (4096,7168) + masked 16x256 (4096,7168) + "
-                 "masked 16x256 (7168,2048), one call each per step")
+WORKLOAD_DESC = ("dense 128x128x512 + decode 64x2112x7168 + prefill 4096x7168x2048 + "
+                 "prefill 256x7168x2048 + contiguous 8 experts (4096,7168) + "
+                 "masked 16x256 (4096,7168) + masked 16x256 (7168,2048), one call each per step")
+# launch-latency-bound: reported, not a roofline target
+LATENCY_BOUND = {"dense_128x128x512"}
 
 
 def log(*a):
@@ -77,19 +83,76 @@ def measured_peaks() -> dict:
 # ---------------------------------------------------------------- workloads
 
 
+def shard_range(n: int, rank: int, world: int) -> tuple[int, int]:
+    """Balanced contiguous share [lo, hi) of n units for `rank` of `world`."""
+    return n * rank // world, n * (rank + 1) // world
+
+
+def shard_problem(prob, rank: int, world: int):
+    """`rank`'s independent part of a workload: no data moves between ranks,
+    and the ranks' outputs, put side by side, are the whole problem's output.
+
+    dense:       a range of 128-column blocks of N (the rows of B and sb of
+                 those blocks, all of A); D's columns of those blocks.
+    contiguous:  a range of experts: their 128-aligned row segments of A (and
+                 sa columns, m_indices renumbered from 0), their B and sb.
+    masked:      a range of groups.
+    A rank whose range is empty gets a problem with no rows or columns.
+    """
+    if world == 1:
+        return prob
+    if isinstance(prob, inputs.DenseProblem):
+        nb = inputs.ceil_div(prob.N, 128)
+        b0, b1 = shard_range(nb, rank, world)
+        c0, c1 = 128 * b0, min(prob.N, 128 * b1)
+        return inputs.DenseProblem(prob.M, max(0, c1 - c0), prob.K, prob.a, prob.sa,
+                                   prob.b[c0:c1].contiguous(), prob.sb[b0:b1].contiguous(),
+                                   prob.seed)
+    if isinstance(prob, inputs.ContiguousProblem):
+        e0, e1 = shard_range(prob.num_groups, rank, world)
+        padded = [inputs.ceil_div(c, inputs.M_ALIGNMENT_CONTIGUOUS) * inputs.M_ALIGNMENT_CONTIGUOUS
+                  for c in prob.counts]
+        offs = np.concatenate([[0], np.cumsum(padded)]).astype(np.int64)
+        r0, r1 = int(offs[e0]), int(offs[e1])
+        mi = prob.m_indices[r0:r1].clone()
+        mi[mi >= 0] -= e0
+        return inputs.ContiguousProblem(e1 - e0, r1 - r0, prob.N, prob.K,
+                                        prob.a[r0:r1].contiguous(),
+                                        prob.sa[:, r0:r1].contiguous(),
+                                        prob.b[e0:e1].contiguous(), prob.sb[e0:e1].contiguous(),
+                                        mi, list(prob.counts[e0:e1]), prob.seed)
+    g0, g1 = shard_range(prob.G, rank, world)
+    return inputs.MaskedProblem(g1 - g0, prob.M_max, prob.N, prob.K, prob.a[g0:g1].contiguous(),
+                                prob.sa[g0:g1].contiguous(), prob.b[g0:g1].contiguous(),
+                                prob.sb[g0:g1].contiguous(), prob.masked_m[g0:g1].contiguous(),
+                                prob.seed)
+
+
+def problem_is_empty(prob) -> bool:
+    if isinstance(prob, inputs.DenseProblem):
+        return prob.M == 0 or prob.N == 0
+    if isinstance(prob, inputs.ContiguousProblem):
+        return prob.num_groups == 0 or prob.M_sum == 0
+    return prob.G == 0
+
+
 class Case:
     """One workload: its device tensors and the C-ABI call that computes it."""
 
-    def __init__(self, name: str, prob):
+    def __init__(self, name: str, prob, rank: int = 0, world: int = 1):
         self.name = name
-        self.prob = prob
         self.kind = type(prob).__name__.replace("Problem", "").lower()
-        self.flops = prob.flops
-        self.bytes = prob.algorithmic_bytes
+        self.whole_flops = prob.flops  # the whole workload (all ranks' shards)
+        self.prob = shard_problem(prob, rank, world)
+        self.empty = problem_is_empty(self.prob)
+        self.flops = self.prob.flops
+        self.bytes = self.prob.algorithmic_bytes
         self.host = {}
         self.dev = {}
 
     def to_device(self):
+        if self.empty:
+            return
         p = self.prob
         self.dev = {"a": p.a.cuda(), "sa": p.sa.cuda(), "b": p.b.cuda(), "sb": p.sb.cuda()}
         if self.kind == "dense":
@@ -103,6 +166,8 @@ class Case:
             self.expected_m = max(1, int(round(float(p.masked_m.float().mean()))))
 
     def pin_host(self):
+        if self.empty:
+            return
         p = self.prob
         self.host = {"a": p.a.pin_memory(), "sa": p.sa.pin_memory(), "b": p.b.pin_memory(),
                      "sb": p.sb.pin_memory(), "d": torch.empty_like(self.dev["d"], device="cpu").pin_memory()}
@@ -115,10 +180,14 @@ class Case:
         return sum(t.numel() * t.element_size() for k, t in self.host.items() if k != "d")
 
     def d2h_bytes(self) -> int:
+        if self.empty:
+            return 0
         return self.host["d"].numel() * self.host["d"].element_size()
 
     def call(self, stream=None):
         import fp8_fine_grained_nt_b200 as fp8
+        if self.empty:
+            return
         d = self.dev
         if self.kind == "dense":
             fp8.gemm_fp8_fp8_bf16_nt(d["a"], d["sa"], d["b"], d["sb"], d["d"], stream=stream)
@@ -130,6 +199,8 @@ class Case:
                                                       d["mm"], self.expected_m, stream=stream)
 
     def e2e_call(self, stream):
+        if self.empty:
+            return
         for k, t in self.host.items():
             if k != "d":
                 self.dev[k].copy_(t, non_blocking=True)
@@ -143,11 +214,11 @@ class Case:
         return (t_tensor, "tensor") if t_tensor >= t_hbm else (t_hbm, "hbm")
 
 
-def make_cases() -> list[Case]:
+def make_cases(rank: int = 0, world: int = 1) -> list[Case]:
     cases = []
     for name in WORKLOAD_NAMES:
         t0 = time.time()
-        cases.append(Case(name, inputs.make_workload(name)))
+        cases.append(Case(name, inputs.make_workload(name), rank, world))
         log(f"generated {name} in {time.time() - t0:.1f}s")
     return cases
 
@@ -417,7 +488,7 @@ def run_gpu(args):
     fp8.load_library()
     peaks = measured_peaks()
 
-    cases = make_cases()
+    cases = make_cases(rank, world)
     for c in cases:
         c.to_device()
     torch.cuda.synchronize()
@@ -458,8 +529,9 @@ def run_gpu(args):
                    for i in range(len(cases))]
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_per_step = elapsed_ms / args.steps
-    step_flops = sum(c.flops for c in cases)
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    # every rank computed its shard of each workload: together, the whole step
+    step_flops = sum(c.whole_flops for c in cases)
+    value = step_flops / (ms_per_step * 1e-3) / 1e12
 
     # e2e: host buffers through the same calls
     for c in cases:
@@ -479,7 +551,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = max_over_ranks(e2e_ms, world)
-    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    e2e_value = step_flops / (e2e_ms * 1e-3) / 1e12
     h2d = sum(c.h2d_bytes() for c in cases)
     d2h = sum(c.d2h_bytes() for c in cases)
     status = fp8.get_device_status()
@@ -488,6 +560,9 @@ def run_gpu(args):
 
     per_shape = {}
     for c, ms in zip(cases, per_case_ms):
+        if c.empty:
+            per_shape[c.name] = {"empty_shard": True}
+            continue
         t_roof, bound = c.roofline_time_s(peaks)
         tflops = c.flops / (ms * 1e-3) / 1e12
         cfg = fp8.select_config(
@@ -503,7 +578,10 @@ def run_gpu(args):
             "frac_of_nominal_fp8": round(tflops / NOMINAL_FP8_TFLOPS, 4),
             "flop": c.flops, "bytes": c.bytes,
             "tile": f"{cfg['block_m']}x{cfg['block_n']}", "stages": cfg["stages"],
+            "split": cfg["split"], "swap_ab": cfg["swap_ab"],
         }
+        if c.name in LATENCY_BOUND:
+            per_shape[c.name]["note"] = "launch-latency bound: reported, not a roofline target"
 
     # dominant kernel: the case with the largest share of step time
     dom_i = int(np.argmax(per_case_ms))
@@ -534,12 +612,14 @@ def run_gpu(args):
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
-            "data": "synthetic",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "fp8_e4m3", "data": "synthetic",
             "config": {"workload": WORKLOAD_DESC,
                        "l2": "each step streams ~1.6 GB of distinct operands (> 126 MB L2); "
                              "every call's operands are evicted by the rest of the step",
-                       "parallelism": f"replicas x{world} (independent problems per GPU)"},
+                       "parallelism": (f"{world} ranks, each an independent shard of every "
+                                       "workload (dense: blocks of N; contiguous: experts; "
+                                       "masked: groups)" if world > 1 else "1 GPU")},
             "per_shape": per_shape,
             "roofline": {"kernel": dom.name, "bound": bound, "achieved": round(achieved, 2),
                          "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
@@ -550,7 +630,7 @@ def run_gpu(args):
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": len(cases) * args.steps,
+            "gpu_launches": sum(1 for c in cases if not c.empty) * args.steps,
             "clocks": clock_info,
             "next_rows": next_rows,
         }
@@ -576,9 +656,28 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        return spawn_ranks(args)
+    if world_env is not None and int(world_env) != args.gpus:
+        log(f"--gpus {args.gpus} does not match WORLD_SIZE={world_env}")
+        return 2
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
+
+
+def spawn_ranks(args) -> int:
+    """Run this script as `args.gpus` ranks on this node (torch.distributed.run,
+    rendezvous on 127.0.0.1); rank 0 prints the JSON line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.run(cmd).returncode
 
 
 if __name__ == "__main__":

@@ -34,6 +34,7 @@ __all__ = [
     "selftest_wait_timeout",
     "select_config",
     "force_config",
+    "force_swap_ab",
     "status_string",
     "KIND_DENSE",
     "KIND_CONTIGUOUS",
@@ -60,7 +61,8 @@ class DgConfig(ctypes.Structure):
                 ("stages", ctypes.c_int),
                 ("num_tiles", ctypes.c_int), ("grid", ctypes.c_int),
                 ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int),
-                ("split", ctypes.c_int), ("cta_pair", ctypes.c_int)]
+                ("split", ctypes.c_int), ("cta_pair", ctypes.c_int),
+                ("swap_ab", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -97,6 +99,7 @@ def load_library():
         lib.dg_get_device_status.argtypes = [P]
         lib.dg_select_config.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(DgConfig)]
         lib.dg_force_config.argtypes = [I, I, I, I]
+        lib.dg_force_swap_ab.argtypes = [I]
         _lib = lib
         return lib
 
@@ -295,3 +298,9 @@ def force_config(block_m: int = 0, block_n: int = 0, split: int = 0, cta_pair: i
     for later calls.  For tests."""
     _check(load_library().dg_force_config(int(block_m), int(block_n), int(split),
                                           int(cta_pair)), "dg_force_config")
+
+
+def force_swap_ab(mode: int = 0) -> None:
+    """Small-M kernel choice for later dense calls: 0 = automatic (M <= 128
+    uses it), 1 = never, 2 = wherever it applies.  For tests."""
+    _check(load_library().dg_force_swap_ab(int(mode)), "dg_force_swap_ab")

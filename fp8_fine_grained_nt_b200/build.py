@@ -1,8 +1,9 @@
 """Build libfp8nt.so in-tree with nvcc for sm_100a (ahead of time, no JIT).
 
 Compiles csrc/api.cu and one object per kernel shape listed in
-csrc/kernels.def (csrc/instance.cu with -DFP8NT_MW / -DFP8NT_BN / -DFP8NT_PAIR / -DFP8NT_SCALAR), in
-parallel, then links them with the static CUDA runtime.  ptxas's resource
+csrc/kernels.def (csrc/instance.cu with -DFP8NT_MW / -DFP8NT_BN / -DFP8NT_PAIR / -DFP8NT_SCALAR)
+and per small-M kernel listed in csrc/skinny.def (csrc/instance_skinny.cu with
+-DFP8NT_SKINNY_MN), in parallel, then links them with the static CUDA runtime.  ptxas's resource
 report is checked for every kernel: the kernels rebalance registers between
 warpgroups with setmaxnreg, which is only safe when each kernel is launched
 with exactly the per-thread register count that split assumes, and spills are
@@ -52,6 +53,17 @@ def kernel_list() -> list[tuple[int, int, int, int]]:
             if m:
                 shapes.append(tuple(int(m.group(i)) for i in range(1, 5)))
     return shapes
+
+
+def skinny_list() -> list[int]:
+    """MN of every small-M dense kernel listed in csrc/skinny.def."""
+    mns = []
+    with open(os.path.join(CSRC, "skinny.def")) as f:
+        for line in f:
+            m = re.match(r"\s*FP8NT_SKINNY\(\s*(\d+)\s*\)", line)
+            if m:
+                mns.append(int(m.group(1)))
+    return mns
 
 
 def kernel_shapes() -> list[tuple[int, int, int]]:
@@ -128,6 +140,10 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -
         tasks.append((os.path.join(CSRC, "instance.cu"), os.path.join(BUILD_DIR, f"kernel_{tag}.o"),
                       [f"-DFP8NT_MW={mw}", f"-DFP8NT_BN={bn}", f"-DFP8NT_PAIR={pair}",
                        f"-DFP8NT_SCALAR={scalar}"], tag))
+    for mn in skinny_list():
+        tasks.append((os.path.join(CSRC, "instance_skinny.cu"),
+                      os.path.join(BUILD_DIR, f"skinny_mn{mn}.o"), [f"-DFP8NT_SKINNY_MN={mn}"],
+                      f"skinny_mn{mn}"))
     notes = []
     with ThreadPoolExecutor(max_workers=jobs) as pool:
         futures = [(t, pool.submit(_compile, t[0], t[1], t[2])) for t in tasks]

@@ -36,6 +36,21 @@ const Candidate kCandidates[] = {
 };
 constexpr int kNumCandidates = sizeof(kCandidates) / sizeof(kCandidates[0]);
 
+// Small-M dense kernels (D^T tiles of 128 rows of B x MN rows of A).
+struct SkinnyCandidate {
+    int mn;
+    SkinnyLaunchFn launch;
+    SkinnyCapacityFn capacity;
+};
+
+const SkinnyCandidate kSkinny[] = {
+#define FP8NT_SKINNY(mn) {mn, launch_skinny_mn##mn, skinny_capacity_mn##mn},
+#include "skinny.def"
+#undef FP8NT_SKINNY
+};
+constexpr int kNumSkinny = sizeof(kSkinny) / sizeof(kSkinny[0]);
+static_assert(kNumSkinny <= 8, "the device capacity cache holds 8 small-M kernels");
+
 constexpr int kDefaultSms = 148;           // B200
 constexpr int kDefaultMaxSmem = 232448;    // 227 KB opt-in per block on sm_100
 constexpr int kMaxStages = 12;
@@ -48,8 +63,17 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull; // 2 s per pipeline wait
 
 // The device status word.  Host code must not take this symbol's address
 // directly: its device address is fetched per device with
-// cudaGetSymbolAddress and passed to the kernels.
+// cudaGetSymbolAddress and passed to the kernels.  The snapshot word receives
+// the status word's value when dg_get_device_status clears it.
 __device__ unsigned int g_status_word;
+__device__ unsigned int g_status_snapshot;
+
+__global__ void status_exchange_kernel(unsigned int *status, unsigned int *snapshot)
+{
+    *snapshot = atomicExch(status, 0u);
+}
+
+std::mutex g_status_mutex;
 
 struct DeviceInfo {
     bool ready;
@@ -58,6 +82,10 @@ struct DeviceInfo {
     int cc_minor;
     int max_smem;
     unsigned int *status;
+    unsigned int *status_snapshot;
+    // clusters of `split` small-M CTAs the device holds at once (0 = not yet
+    // asked, -1 = the query failed), per kernel of kSkinny
+    std::atomic<int> skinny_cap[8][SKINNY_MAX_SPLIT + 1];
 };
 
 constexpr int kMaxDevices = 64;
@@ -69,8 +97,12 @@ std::mutex g_mutex;
 std::atomic<int> g_num_sms_limit{0};
 std::atomic<uint32_t> g_forced{0};
 
+// swap: 0 = automatic, 1 = never the small-M (swap-AB) kernel, 2 = always
+// where it applies (dense calls with M <= 128).
+std::atomic<int> g_forced_swap{0};
+
 struct Forced {
-    int bm, bn, split, pair;
+    int bm, bn, split, pair, swap;
 };
 
 uint32_t pack_forced(int bm, int bn, int split, int pair)
@@ -82,7 +114,7 @@ Forced forced_config()
 {
     const uint32_t w = g_forced.load(std::memory_order_relaxed);
     return Forced{(int)(w & 0x3FF), (int)((w >> 10) & 0x3FF), (int)((w >> 20) & 0xF),
-                  (int)((w >> 24) & 0x3)};
+                  (int)((w >> 24) & 0x3), g_forced_swap.load(std::memory_order_relaxed)};
 }
 
 int device_info(DeviceInfo **out)
@@ -105,6 +137,9 @@ int device_info(DeviceInfo **out)
         if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess)
             return DG_ERR_CUDA;
         d.status = static_cast<unsigned int *>(addr);
+        if (cudaGetSymbolAddress(&addr, g_status_snapshot) != cudaSuccess)
+            return DG_ERR_CUDA;
+        d.status_snapshot = static_cast<unsigned int *>(addr);
         d.ready = true;
     }
     *out = &d;
@@ -371,6 +406,7 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     cfg->num_tiles = (int)tiles;
     cfg->split = best_split;
     cfg->cta_pair = best->pair ? 2 : 1;
+    cfg->swap_ab = 0;
     if (best_split > 1)
         cfg->grid = (int)tiles * best_split; // one tile per cluster
     else if (best->pair)
@@ -388,6 +424,166 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     return DG_OK;
 }
 
+// ------------------------------------------------------------------ small M
+
+// Dynamic shared memory of a small-M CTA is never below this, so that one CTA
+// runs per SM (each allocates the SM's whole tensor memory) and the cluster
+// capacity does not depend on K.
+constexpr int kSkinnyMinSmem = 116 * 1024;
+
+// Clusters of `split` CTAs (one per SM) that can run at once, when the device
+// has not been asked: a cluster does not span a GPC, and B200's 148 SMs form
+// 8 GPCs of at least 18 SMs; a lowered SM bound caps it too.
+int cluster_capacity_model(int split, int sms)
+{
+    if (split <= 1)
+        return sms;
+    const int by_gpc = 8 * (18 / split);
+    const int by_sms = sms / split;
+    const int cap = by_gpc < by_sms ? by_gpc : by_sms;
+    return cap > 0 ? cap : 1;
+}
+
+// Cycle estimate of a small-M choice: waves of clusters, each CTA streaming
+// its share of K blocks at the slowest of (a) the four MMAs of a K block (at
+// least ~64 cycles each for one issuing thread, ~75 at N = 128), (b) its share
+// of the HBM bandwidth (~3300 B/clk at the boost clock) for 16 KB of B per K
+// block, (c) one SM's TMA ingest (~110 B/clk); plus set-up and, with a
+// cluster, the reduction of the partial tiles through distributed shared
+// memory.
+double skinny_cycles(int N, int K, int mn, int split, int cap)
+{
+    const long tiles = ceil_div(N, SKINNY_TILE_N);
+    const int nkb = K / 128;
+    const long waves = (tiles + cap - 1) / cap;
+    const long active = (tiles < cap ? tiles : cap) * (long)split;
+    const int cnt = ceil_div(nkb, split);
+    const double t_mma = 4.0 * (mn <= 64 ? 64.0 : 75.0);
+    const double t_hbm = 128.0 * 128.0 * (double)active / 3300.0;
+    const double t_tma = (128.0 + mn) * 128.0 / 110.0;
+    double t_kb = t_mma > t_hbm ? t_mma : t_hbm;
+    t_kb = t_kb > t_tma ? t_kb : t_tma;
+    return (double)waves * (1200.0 + cnt * t_kb + (split > 1 ? 800.0 + 100.0 * split : 300.0));
+}
+
+struct SkinnyChoice {
+    const SkinnyCandidate *cand;
+    int cand_index;
+    SkinnyParams plan; // sizes, split, stages and shared-memory offsets
+    int smem_bytes;
+};
+
+// Shared-memory plan of a small-M kernel: as many operand stages as fit, up to
+// the CTA's number of K blocks.
+bool skinny_plan(const Problem &pb, int mn, int split, int max_smem, SkinnyParams *out)
+{
+    SkinnyParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = pb.M;
+    p.N = pb.N;
+    p.K = pb.K;
+    p.nkb = pb.K / 128;
+    p.n_tiles = ceil_div(pb.N, SKINNY_TILE_N);
+    p.split = split;
+    p.kb_max = ceil_div(p.nkb, split);
+    int st = p.kb_max < DONE_RING ? p.kb_max : DONE_RING;
+    for (; st >= 1; --st) {
+        make_skinny_plan(p, mn, st);
+        if ((int)p.total + 1024 <= max_smem)
+            break;
+    }
+    if (st < 1 || (st < 2 && p.kb_max > 1))
+        return false;
+    *out = p;
+    return true;
+}
+
+// Capacity of the device (queried once per kernel and cluster size), or the
+// GPC model when no device is given or the query fails.
+int skinny_capacity(DeviceInfo *dev, int idx, int split, int sms)
+{
+    const int model = cluster_capacity_model(split, sms);
+    if (!dev)
+        return model;
+    int c = dev->skinny_cap[idx][split].load(std::memory_order_relaxed);
+    if (c == 0) {
+        c = kSkinny[idx].capacity(split, kSkinnyMinSmem);
+        dev->skinny_cap[idx][split].store(c > 0 ? c : -1, std::memory_order_relaxed);
+    }
+    if (c <= 0)
+        return model;
+    // a lowered SM bound (set_num_sms) caps the device's own figure
+    const int by_sms = sms / split > 0 ? sms / split : 1;
+    return c < by_sms ? c : by_sms;
+}
+
+// Small-M kernel for a dense call: the smallest MN >= M, and the cluster size
+// (CTAs sharing a tile's K range) with the lowest estimate.
+int choose_skinny(const Problem &pb, int sms, int max_smem, DeviceInfo *dev, SkinnyChoice *out)
+{
+    const Forced forced = forced_config();
+    int idx = -1;
+    for (int i = 0; i < kNumSkinny; ++i)
+        if (kSkinny[i].mn >= pb.M && (idx < 0 || kSkinny[i].mn < kSkinny[idx].mn))
+            idx = i;
+    if (idx < 0)
+        return DG_ERR_UNSUPPORTED_SHAPE;
+    const int nkb = pb.K / 128;
+    double best = 0;
+    bool found = false;
+    for (int split = 1; split <= SKINNY_MAX_SPLIT; ++split) {
+        if (forced.split ? split != forced.split : split > nkb)
+            continue;
+        SkinnyParams p;
+        if (!skinny_plan(pb, kSkinny[idx].mn, split, max_smem, &p))
+            continue;
+        const int cap = skinny_capacity(dev, idx, split, sms);
+        const double cost = skinny_cycles(pb.N, pb.K, kSkinny[idx].mn, split, cap);
+        if (!found || cost < best * (1 - 1e-9)) {
+            found = true;
+            best = cost;
+            out->cand = &kSkinny[idx];
+            out->cand_index = idx;
+            out->plan = p;
+            const int need = (int)p.total + 1024;
+            out->smem_bytes = need > kSkinnyMinSmem ? need : kSkinnyMinSmem;
+        }
+    }
+    return found ? DG_OK : DG_ERR_UNSUPPORTED_SHAPE;
+}
+
+// Dense calls with M <= 128 take the small-M kernel, unless the test hooks
+// turn it off or pin a tile shape or CTA pairs of the other kernels.
+bool use_skinny(const Problem &pb)
+{
+    if (pb.kind != DG_KIND_DENSE || pb.M > SKINNY_MAX_M)
+        return false;
+    if ((long)ceil_div(pb.N, SKINNY_TILE_N) > 65535)
+        return false; // grid.y limit
+    const Forced f = forced_config();
+    if (f.swap != 0)
+        return f.swap == 2;
+    return f.bm == 0 && f.pair != 2;
+}
+
+void skinny_config(const SkinnyChoice &c, dg_config *cfg)
+{
+    memset(cfg, 0, sizeof(*cfg));
+    cfg->block_m = c.cand->mn;
+    cfg->block_n = SKINNY_TILE_N;
+    cfg->stages = c.plan.stages;
+    cfg->num_tiles = c.plan.n_tiles;
+    cfg->grid = c.plan.n_tiles * c.plan.split;
+    cfg->smem_bytes = c.smem_bytes;
+    const int mn = c.cand->mn;
+    const int nbuf = 512 / mn < MAX_TMEM_BUFS ? 512 / mn : MAX_TMEM_BUFS;
+    const int need = nbuf * mn;
+    cfg->tmem_cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
+    cfg->split = c.plan.split;
+    cfg->cta_pair = 1;
+    cfg->swap_ab = 1;
+}
+
 int effective_sms(const DeviceInfo *d)
 {
     int n = d ? d->sm_count : kDefaultSms;
@@ -400,7 +596,7 @@ int effective_sms(const DeviceInfo *d)
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_common(const void *A, const float *sa, const void *B, const float *sb, void *D, int M,
-                 int N, int K)
+                 int N, int K, bool scalar_scales = false)
 {
     if (M < 0 || N < 0 || K < 0)
         return DG_ERR_INVALID_ARGUMENT;
@@ -410,9 +606,57 @@ int check_common(const void *A, const float *sa, const void *B, const float *sb,
         return DG_OK;
     if (!A || !sa || !B || !sb || !D)
         return DG_ERR_INVALID_ARGUMENT;
-    if (!aligned16(A) || !aligned16(sa) || !aligned16(B) || !aligned16(sb) || !aligned16(D))
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D))
+        return DG_ERR_MISALIGNED;
+    // per-tensor scales are single FP32 values read as scalars: 4-byte
+    // alignment; block scales are tensors read by TMA / vector copies: 16
+    const uintptr_t scale_align = scalar_scales ? 3u : 15u;
+    if ((reinterpret_cast<uintptr_t>(sa) & scale_align) || (reinterpret_cast<uintptr_t>(sb) & scale_align))
         return DG_ERR_MISALIGNED;
     return DG_OK;
+}
+
+// Dense call with M <= 128 through the small-M kernel.
+int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const void *A, const float *sa,
+               const void *B, const float *sb, void *D, cudaStream_t stream)
+{
+    SkinnyChoice ch;
+    int st = choose_skinny(pb, sms, dev->max_smem, dev, &ch);
+    if (st != DG_OK)
+        return st;
+    CUtensorMap tmap_a, tmap_b;
+    // A: [M][K] bytes, box MN rows x 128 (rows past M are zero-filled); B:
+    // [N][K] bytes, box 128 rows x 128
+    if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, pb.M, pb.K, 128,
+                           (uint32_t)ch.cand->mn, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+        return st;
+    if ((st = make_tmap_2d(&tmap_b, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, pb.N, pb.K, 128,
+                           SKINNY_TILE_N, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
+        return st;
+    SkinnyParams p = ch.plan;
+    p.sa = sa;
+    p.ld_sa = get_tma_aligned_size(pb.M, 4);
+    p.sb = sb;
+    p.D = static_cast<uint16_t *>(D);
+    p.status = dev->status;
+    p.timeout_ns = wait_timeout_ns();
+    // persistent clusters: no more than the SM bound (and the device) holds
+    const int cap = skinny_capacity(dev, ch.cand_index, p.split, sms);
+    const int by_sms = sms / p.split > 0 ? sms / p.split : 1;
+    int clusters = p.n_tiles;
+    if (clusters > cap)
+        clusters = cap;
+    if (clusters > by_sms)
+        clusters = by_sms;
+    SkinnyLaunchArgs args;
+    args.tmap_a = &tmap_a;
+    args.tmap_b = &tmap_b;
+    args.params = &p;
+    args.split = p.split;
+    args.n_tiles = clusters;
+    args.smem_bytes = ch.smem_bytes;
+    args.stream = stream;
+    return ch.cand->launch(args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
 // Shared launch path for the three forms.
@@ -424,6 +668,8 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     if (st != DG_OK)
         return st;
     const int sms = effective_sms(dev);
+    if (use_skinny(pb))
+        return run_skinny(pb, dev, sms, A, sa, B, sb, D, stream);
     const Candidate *cand = nullptr;
     dg_config cfg;
     SmemPlan plan;
@@ -542,7 +788,7 @@ int gemm_fp8_fp8_bf16_nt_per_tensor(const void *A, const float *scale_a, const v
                                     const float *scale_b, void *D, int M, int N, int K,
                                     dg_stream_t stream)
 {
-    int st = check_common(A, scale_a, B, scale_b, D, M, N, K);
+    int st = check_common(A, scale_a, B, scale_b, D, M, N, K, true);
     if (st != DG_OK || M == 0 || N == 0)
         return st;
     Problem pb{DG_KIND_DENSE_PER_TENSOR, M, N, K, 1, 0};
@@ -683,16 +929,18 @@ int dg_get_device_status(dg_stream_t stream)
     int st = device_info(&dev);
     if (st != DG_OK)
         return st;
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    // One thread swaps the status word for zero (so a bit set by a kernel on
+    // another stream is either reported now or kept for the next call, never
+    // lost) and leaves the old value in the snapshot word; host threads take
+    // turns, so each reads its own snapshot.
+    std::lock_guard<std::mutex> lock(g_status_mutex);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    status_exchange_kernel<<<1, 1, 0, s>>>(dev->status, dev->status_snapshot);
+    if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
         return DG_ERR_CUDA;
     unsigned int word = 0;
-    if (cudaMemcpy(&word, dev->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    if (cudaMemcpy(&word, dev->status_snapshot, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
         return DG_ERR_CUDA;
-    if (word != 0) {
-        const unsigned int zero = 0;
-        if (cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
-            return DG_ERR_CUDA;
-    }
     if (word & DEVERR_TIMEOUT)
         return DG_ERR_DEVICE_TIMEOUT;
     if (word & DEVERR_BAD_INDEX)
@@ -713,14 +961,30 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
     int sms = num_sms > 0 ? num_sms : (limit > 0 ? limit : kDefaultSms);
     const bool one_group = kind == DG_KIND_DENSE || kind == DG_KIND_DENSE_PER_TENSOR;
     Problem pb{kind, M, N, K, one_group ? 1 : num_groups, expected_m};
+    if (use_skinny(pb)) {
+        SkinnyChoice ch;
+        const int st = choose_skinny(pb, sms, kDefaultMaxSmem, nullptr, &ch);
+        if (st != DG_OK)
+            return st;
+        skinny_config(ch, out);
+        const int cap = cluster_capacity_model(ch.plan.split, sms);
+        const int by_sms = sms / ch.plan.split > 0 ? sms / ch.plan.split : 1;
+        int clusters = ch.plan.n_tiles < cap ? ch.plan.n_tiles : cap;
+        clusters = clusters < by_sms ? clusters : by_sms;
+        out->grid = clusters * ch.plan.split;
+        return DG_OK;
+    }
     const Candidate *cand = nullptr;
     SmemPlan plan;
-    return choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);
+    const int st = choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);
+    if (st == DG_OK)
+        out->swap_ab = 0;
+    return st;
 }
 
 int dg_force_config(int block_m, int block_n, int split, int cta_pair)
 {
-    if (split < 0 || split > kMaxSplit || (split & (split - 1)) != 0)
+    if (split < 0 || split > kMaxSplit)
         return DG_ERR_UNSUPPORTED_SHAPE;
     if (cta_pair < 0 || cta_pair > 2)
         return DG_ERR_UNSUPPORTED_SHAPE;
@@ -737,6 +1001,14 @@ int dg_force_config(int block_m, int block_n, int split, int cta_pair)
         }
     }
     return DG_ERR_UNSUPPORTED_SHAPE;
+}
+
+int dg_force_swap_ab(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return DG_ERR_INVALID_ARGUMENT;
+    g_forced_swap.store(mode, std::memory_order_relaxed);
+    return DG_OK;
 }
 
 } // extern "C"

@@ -719,11 +719,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // order, so a slot is awaited at its first K block and released
             // after its last (rows past M read the zero fill and are never
             // stored)
+            // (returns false if the wait for a slot failed: the caller stops)
             auto scales = [&](int kb, float &s_lo, float &s_hi) {
                 const int gpos = (kb - kb_lo) % T::SA_GROUP;
                 const uint32_t gs = sa_it & 1;
-                if (gpos == 0)
-                    wait_bar_warp(&sa_full[gs], (sa_it >> 1) & 1, abort_flag, p);
+                if (gpos == 0 && !wait_bar_warp(&sa_full[gs], (sa_it >> 1) & 1, abort_flag, p))
+                    return false;
                 const float sa_v = sa_ring[gs * (SA_SLOT_BYTES / 4) + gpos * T::SA_ROWS + row_in_tile];
                 if (gpos == T::SA_GROUP - 1 || kb == kb_hi - 1) {
                     __syncwarp();
@@ -732,7 +733,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ++sa_it;
                 }
                 s_lo = sa_v * sbt[lo * pitch + kb];
-                s_hi = sa_v * sbt[(lo + 1) * pitch + kb];
+                // the next scale block exists only where the columns cross into it
+                s_hi = split ? sa_v * sbt[(lo + 1) * pitch + kb] : s_lo;
+                return true;
             };
 #pragma unroll
             for (int c = 0; c < NC; ++c)
@@ -791,7 +794,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int j = 0; j < G; ++j) {
                         if (j < cnt) {
                             float s_lo, s_hi;
-                            scales(kb0 + j, s_lo, s_hi);
+                            if (!scales(kb0 + j, s_lo, s_hi)) {
+                                if (more && active)
+                                    tmem_wait64(nxt); // no load left in flight
+                                return false;
+                            }
                             if (active) {
                                 if (split)
                                     fma_all_p<NC, true>(acc, &cur[j * NC], s_lo, s_hi, t_split);
@@ -836,7 +843,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (active)
                         tmem_issue<B0>(buf_addr(kb_it), r);
                     float s_lo, s_hi;
-                    scales(kb, s_lo, s_hi);
+                    if (!scales(kb, s_lo, s_hi)) {
+                        if (active)
+                            tmem_wait64(r); // no load left in flight
+                        ok = false;
+                        break;
+                    }
                     if (active) {
                         tmem_wait64(r);
                         fma_range_any<NC, 0, B0>(acc, r, s_lo, s_hi, t_split, split);

@@ -118,4 +118,56 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     return p;
 }
 
+// ---------------------------------------------------------------- skinny kernel
+// Dense GEMM with few rows of A (M <= 128, decode-shaped calls), computed as
+// D^T tiles: 128 rows of B per tile on the MMA's M side and the rows of A,
+// zero-padded to MN, on its N side (kernel_skinny.cuh).
+
+constexpr int SKINNY_THREADS = 256;      // warps 0-3: roles, warps 4-7: epilogue
+constexpr int SKINNY_TILE_N = 128;       // rows of B (columns of D) per tile
+constexpr int SKINNY_MAX_SPLIT = 8;      // CTAs per cluster sharing a tile's K range
+constexpr int SKINNY_MAX_M = 128;
+
+struct SkinnyParams {
+    int M;          // rows of A and D (<= MN of the kernel)
+    int N;
+    int K;
+    int nkb;        // K / 128
+    int n_tiles;    // ceil(N / 128)
+    int split;      // CTAs of a cluster that share one tile, each a contiguous K range
+    int kb_max;     // K blocks of the largest share: ceil(nkb / split)
+    int stages;     // operand ring depth
+    uint32_t stage_bytes; // 128 x 128 B of B, then MN x 128 B of A
+    uint32_t region;      // operand ring, reused for the FP32 partial tile at the end
+    uint32_t off_sa;      // LHS scales of the CTA's K range: kb_max x MN FP32
+    uint32_t off_sb;      // RHS scales of the tile's 128-row block: kb_max FP32
+    uint32_t off_bars;
+    uint32_t off_misc;    // TMEM base address, abort flag
+    uint32_t total;       // bytes, excluding the 1024 B alignment slack
+    const float *sa;      // [K/128][ld_sa]
+    int ld_sa;
+    const float *sb;      // [ceil(N/128)][K/128]
+    uint16_t *D;          // [M][N] BF16 bits
+    unsigned int *status;
+    uint64_t timeout_ns;
+};
+
+// Barriers of the skinny kernel: full per stage, "K block done" ring, TMEM
+// buffer released (ring), scales loaded, all MMAs done.
+constexpr int SKINNY_NUM_BARS_FIXED = DONE_RING + MAX_TMEM_BUFS + 2;
+
+__host__ __device__ inline void make_skinny_plan(SkinnyParams &p, int mn, int stages)
+{
+    p.stages = stages;
+    p.stage_bytes = (uint32_t)(SKINNY_TILE_N + mn) * BLOCK_K;
+    const uint32_t ring = p.stage_bytes * (uint32_t)stages;
+    const uint32_t red = (uint32_t)mn * SKINNY_TILE_N * 4u;
+    p.region = ring > red ? ring : red;
+    p.off_sa = align_up_u32(p.region, 128);
+    p.off_sb = p.off_sa + (uint32_t)p.kb_max * (uint32_t)mn * 4u;
+    p.off_bars = align_up_u32(p.off_sb + (uint32_t)p.kb_max * 4u, 8);
+    p.off_misc = align_up_u32(p.off_bars + 8u * (uint32_t)(stages + SKINNY_NUM_BARS_FIXED), 16);
+    p.total = p.off_misc + 16;
+}
+
 } // namespace fp8nt

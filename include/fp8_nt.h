@@ -17,7 +17,8 @@
  * Pointers.  Every pointer is CUDA device memory owned by the caller.  The
  *   library never allocates, frees or keeps a reference to it after the call
  *   returns; it reads A, sa, B, sb (and m_indices / masked_m) and writes D.
- *   Every pointer must be 16-byte aligned.
+ *   Every pointer must be 16-byte aligned (except the two single-value
+ *   scales of gemm_fp8_fp8_bf16_nt_per_tensor: 4-byte aligned).
  * Element types.  A and B hold E4M3 bytes (1 sign, 4 exponent bits with bias
  *   7, 3 mantissa bits; 0x7F/0xFF are NaN).  sa and sb are IEEE FP32.  D is
  *   BF16 (stored as uint16).
@@ -73,7 +74,8 @@ int gemm_fp8_fp8_bf16_nt(const void *A, const float *sa, const void *B, const fl
  * accumulated in FP32 over the whole K range in tensor memory (no per-block
  * promotion is needed when every block has the same scale) and rounded to
  * BF16 (RNE).  scale_a and scale_b point to ONE FP32 value each, in device
- * memory (read by the kernel, so a CUDA graph can update them).  A, B, D and
+ * memory (read by the kernel, so a CUDA graph can update them), 4-byte
+ * aligned (an element of a larger scales tensor is fine).  A, B, D and
  * the shape rules are as for gemm_fp8_fp8_bf16_nt. */
 int gemm_fp8_fp8_bf16_nt_per_tensor(const void *A, const float *scale_a, const void *B,
                                     const float *scale_b, void *D, int M, int N, int K,
@@ -159,9 +161,13 @@ int dg_selftest_wait_timeout(int timeout_us, dg_stream_t stream);
 /* Static description of a dg_status value. */
 const char *dg_status_string(int status);
 
-/* Synchronises `stream`, then returns and clears the device status word
- * (DG_OK, DG_ERR_DEVICE_TIMEOUT or DG_ERR_DEVICE_BAD_INDEX), or DG_ERR_CUDA if
- * the synchronisation itself failed. */
+/* Reads and clears the device status word in one atomic exchange, enqueued
+ * on `stream` (so it follows the work enqueued there), synchronises `stream`
+ * and returns what it read: DG_OK, DG_ERR_DEVICE_TIMEOUT or
+ * DG_ERR_DEVICE_BAD_INDEX; DG_ERR_CUDA if the launch or the synchronisation
+ * failed.  A bit set meanwhile by a kernel on another stream is reported by
+ * this call or by the next one, never dropped.  Host threads calling it take
+ * turns. */
 int dg_get_device_status(dg_stream_t stream);
 
 /* Tile configuration chosen for a call (host logic; no GPU needed). */
@@ -178,6 +184,12 @@ typedef struct dg_config {
     int cta_pair;   /* 2: a cluster of two CTAs computes each 256-row tile with
                        tcgen05 cta_group::2 MMAs (each CTA loads its own 128 rows
                        of A and half of the B tile); 1: one CTA per tile */
+    int swap_ab;    /* 1: the small-M dense kernel (M <= 128): each tile is
+                       128 rows of B (block_n = 128 columns of D) against all
+                       rows of A zero-padded to block_m, computed as D^T with
+                       B in the MMA's 128-row slot; split CTAs of a cluster
+                       share the tile's K range and reduce through distributed
+                       shared memory.  0: the kernels described above. */
 } dg_config;
 
 enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2, DG_KIND_DENSE_PER_TENSOR = 3 };
@@ -195,11 +207,18 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
 
 /* Test hook: pin block_m / block_n, the split-K factor and the CTA-pair mode
  * for later calls (0, 0 restores automatic tile choice; split 0 = automatic,
- * 1 = no split, 2, 4 or 8 = that many CTAs per tile, used only where split-K
- * applies; cta_pair 0 = automatic, 1 = one CTA per tile, 2 = CTA pairs).
- * Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that shape is built, the
- * split is not 0, 1, 2, 4 or 8, or cta_pair is not 0, 1 or 2. */
+ * 1 = no split, 2..8 = that many CTAs per tile, used only where split-K
+ * applies: 2, 4 or 8 for the kernels with 128- or 256-row tiles, any of 1..8
+ * for the small-M kernel; cta_pair 0 = automatic, 1 = one CTA per tile,
+ * 2 = CTA pairs).  block_m / block_n pin the tile of the kernels other than
+ * the small-M one.  Returns DG_ERR_UNSUPPORTED_SHAPE if no kernel of that
+ * shape is built, the split is outside 0..8, or cta_pair is not 0, 1 or 2. */
 int dg_force_config(int block_m, int block_n, int split, int cta_pair);
+
+/* Test hook: 0 = automatic (dense calls with M <= 128 use the small-M kernel
+ * of dg_config.swap_ab), 1 = never use it, 2 = use it wherever it applies.
+ * Returns DG_OK, or DG_ERR_INVALID_ARGUMENT for another mode. */
+int dg_force_swap_ab(int mode);
 
 #ifdef __cplusplus
 }

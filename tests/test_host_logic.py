@@ -130,6 +130,17 @@ def test_selector_invariants_and_determinism(lib):
         a = fp8.select_config(kind, M, N, K, G, em, 148)
         b = fp8.select_config(kind, M, N, K, G, em, 148)
         assert a == b
+        if a["swap_ab"]:
+            # small-M kernel: dense, M <= 128, tiles of 128 columns of D
+            assert kind == fp8.KIND_DENSE and M <= 128
+            assert a["block_m"] in (16, 32, 64, 128) and a["block_m"] >= M
+            assert a["block_m"] // 2 < M or a["block_m"] == 16
+            assert a["block_n"] == 128 and a["num_tiles"] == -(-N // 128)
+            assert 1 <= a["split"] <= min(8, K // 128)
+            assert a["grid"] % a["split"] == 0 and 1 <= a["grid"] <= 148
+            assert a["stages"] >= min(2, K // 128) and a["smem_bytes"] <= 232448
+            assert a["tmem_cols"] <= 512 and a["cta_pair"] == 1
+            continue
         assert a["block_m"] in (128, 256) and a["block_n"] % 16 == 0
         assert a["cta_pair"] in (1, 2)
         pair = a["cta_pair"] == 2
@@ -149,8 +160,11 @@ def test_selector_invariants_and_determinism(lib):
 
 
 def test_decode_shape_uses_split_k_in_one_wave(lib):
+    """The decode shape runs on the small-M kernel: 17 tiles of 128 columns,
+    each K range split over a cluster, all clusters resident at once."""
     cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)
-    assert cfg["split"] in (2, 4)
+    assert cfg["swap_ab"] == 1 and cfg["block_m"] == 64 and cfg["num_tiles"] == 17
+    assert 2 <= cfg["split"] <= 8
     assert cfg["grid"] == cfg["num_tiles"] * cfg["split"] <= 148
     # large problems never split
     assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["split"] == 1
@@ -164,9 +178,45 @@ def test_forced_split(lib):
         cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)
         assert (cfg["block_n"], cfg["split"]) == (64, 4)
         with pytest.raises(fp8.Fp8NtError):
-            fp8.force_config(128, 64, 3)
+            fp8.force_config(128, 64, 9)
+        # a pinned tile of the 128-row kernels keeps small M off the small-M kernel
+        assert cfg["swap_ab"] == 0
+        # the small-M kernel takes any split of 1..8
+        fp8.force_config(0, 0, 3)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)
+        assert (cfg["swap_ab"], cfg["split"], cfg["grid"]) == (1, 3, 51)
     finally:
         fp8.force_config(0, 0, 0)
+
+
+def test_force_swap_ab(lib):
+    try:
+        fp8.force_swap_ab(1)
+        cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)
+        assert cfg["swap_ab"] == 0 and cfg["block_m"] == 128
+        fp8.force_swap_ab(2)
+        fp8.force_config(128, 64)
+        assert fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)["swap_ab"] == 1
+        # never for M > 128 or the grouped forms
+        assert fp8.select_config(fp8.KIND_DENSE, 129, 2112, 7168, num_sms=148)["swap_ab"] == 0
+        assert fp8.select_config(fp8.KIND_MASKED, 64, 4096, 7168, 4, 32, 148)["swap_ab"] == 0
+        with pytest.raises(fp8.Fp8NtError):
+            fp8.force_swap_ab(3)
+    finally:
+        fp8.force_swap_ab(0)
+        fp8.force_config(0, 0)
+
+
+def test_small_m_kernel_choice(lib):
+    """MN is the smallest built width >= M; split never exceeds the K blocks;
+    a lowered SM bound caps the clusters launched."""
+    for M, mn in ((1, 16), (16, 16), (17, 32), (33, 64), (64, 64), (65, 128), (128, 128)):
+        cfg = fp8.select_config(fp8.KIND_DENSE, M, 4096, 7168, num_sms=148)
+        assert (cfg["swap_ab"], cfg["block_m"]) == (1, mn)
+    cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 256, num_sms=148)
+    assert cfg["split"] <= 2
+    cfg = fp8.select_config(fp8.KIND_DENSE, 64, 65536, 7168, num_sms=16)
+    assert cfg["grid"] <= 16 and cfg["num_tiles"] == 512
 
 
 def test_force_config_rejects_unbuilt_shapes(lib):
@@ -233,6 +283,18 @@ def test_per_tensor_host_checks_and_selection(lib):
     assert g(p, p, p, p, p, 0, 128, 128, None) == 0     # empty
     assert g(p, None, p, p, p, 128, 128, 128, None) == 1
     assert g(p, p, mis, p, p, 128, 128, 128, None) == 2
+    # the two scales are single FP32 values: 4-byte alignment is enough
+    odd = ctypes.c_void_p(0x10002)
+    four = ctypes.c_void_p(0x10004)
+    assert g(p, odd, p, p, p, 128, 128, 128, None) == 2
+    assert g(p, p, p, odd, p, 128, 128, 128, None) == 2
+    import torch
+    if not torch.cuda.is_available():
+        # passes the argument checks; with no device the call then fails on
+        # the device query (never reached with these addresses on a GPU machine)
+        assert g(p, four, p, four, p, 128, 128, 128, None) == 5
+        # block scales still need 16 bytes
+        assert lib.gemm_fp8_fp8_bf16_nt(p, four, p, p, p, 128, 128, 128, None) == 2
     from fp8_fine_grained_nt_b200 import build
     scalar_bns = set(build.scalar_kernel_shapes())
     assert scalar_bns and scalar_bns <= {64, 128, 192, 256}
