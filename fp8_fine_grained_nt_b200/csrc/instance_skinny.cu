@@ -48,18 +48,23 @@ cudaError_t FP8NT_SK_NAME(launch_skinny_mn, FP8NT_SKINNY_MN)(const SkinnyLaunchA
         return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)args.split, (unsigned)args.n_tiles, 1);
-    cfg.blockDim = dim3(SKINNY_THREADS, 1, 1);
+    cfg.blockDim = dim3(SkinnyTraits<FP8NT_SKINNY_MN>::THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)args.smem_bytes;
     cfg.stream = args.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cfg.attrs = attr;
-    cfg.numAttrs = 0;
+    // programmatic dependent launch: the kernel's set-up may overlap the
+    // previous kernel in the stream (it waits for that kernel before touching
+    // global memory)
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 1;
     if (args.split > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)args.split;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.numAttrs = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)args.split;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
     }
     return cudaLaunchKernelEx(&cfg, fp8_gemm_skinny_kernel<FP8NT_SKINNY_MN>, *args.tmap_a, *args.tmap_b,
                               *args.params);
@@ -73,7 +78,7 @@ int FP8NT_SK_NAME(skinny_capacity_mn, FP8NT_SKINNY_MN)(int split, int smem_bytes
     }
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3((unsigned)(split > 0 ? split : 1), 1, 1);
-    q.blockDim = dim3(SKINNY_THREADS, 1, 1);
+    q.blockDim = dim3(SkinnyTraits<FP8NT_SKINNY_MN>::THREADS, 1, 1);
     q.dynamicSmemBytes = (size_t)smem_bytes;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;

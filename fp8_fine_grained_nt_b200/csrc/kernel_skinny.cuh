@@ -15,16 +15,23 @@
 // a shared-memory ring at once (as deep as shared memory allows), one thread
 // issues the MMAs of every K block into its own TMEM buffer (the ring of
 // 512 / MN buffers usually holds the CTA's whole range, so the MMAs never wait
-// for the epilogue), and four epilogue warps promote each partial into FP32
-// registers as it completes.  At the end the CTAs' FP32 partial tiles meet in
-// shared memory; each CTA sums a share of the output in rank order through
-// distributed shared memory (deterministic) and stores it as BF16.
+// for the epilogue), and the epilogue warps promote each partial into FP32
+// registers as it completes.  At the end each CTA owns a share of the output
+// tile: every CTA sends the matching slices of its FP32 partial tile to their
+// owners with bulk copies into the owners' shared memory (the copy engine
+// moves them; completion is counted on the owner's barrier), and each owner
+// sums the slices in rank order (deterministic) and stores them as BF16.
 //
-// Roles (256 threads, one CTA per SM):
-//   warp 0      TMA producer of the B and A tiles (lane 0)
+// Roles (one CTA per SM; 256 threads, 384 for MN = 128):
+//   warp 0      TMA producer of the B tiles (lane 0)
+//   warp 3      TMA producer of the A tiles (lane 0); the two copiers' issue
+//               latencies overlap, each arriving on a stage's barrier with
+//               its own bytes
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warp 2      loads the CTA's LHS and RHS scales into shared memory
-//   warps 4-7   promotion epilogue (TMEM lane quarter = warp - 4)
+//   warp 2      copies the CTA's LHS and RHS scales into shared memory
+//               (asynchronous copies, started at kernel entry)
+//   warps 4..   promotion epilogue: one warpgroup (two for MN = 128, each
+//               with half of the columns); TMEM lane quarter = warp % 4
 #pragma once
 
 #include "kernel.cuh"
@@ -42,10 +49,14 @@ struct SkinnyTraits {
     static constexpr int TMEM_NEED = NBUF * MN;
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                    : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-    // a partial of up to 64 columns fits one register batch: the next K
-    // block's partial is then in flight while the current one is promoted
-    static constexpr bool PREFETCH = MN <= 64;
-    static constexpr int CHUNK = MN <= 64 ? MN : 32; // columns per tcgen05.ld batch
+    // epilogue warpgroups and the columns each thread owns (at most 64)
+    static constexpr int EPI_WGS = MN > 64 ? 2 : 1;
+    static constexpr int COLS = MN / EPI_WGS;
+    static constexpr int THREADS = 128 + 128 * EPI_WGS;
+    // with one warpgroup (256 threads, up to 255 registers each) the next K
+    // block's partial is in flight while the current one is promoted; with
+    // two (384 threads, 168 registers) one partial at a time
+    static constexpr bool PREFETCH = EPI_WGS == 1;
 };
 
 // Ties 16 registers to this point of the instruction stream (no code).
@@ -90,6 +101,15 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi)
     return r;
 }
 
+// 16-byte asynchronous copy global -> shared that reads `src_bytes` (0..16)
+// and zero-fills the rest of the 16 bytes.
+__device__ __forceinline__ void cp_async_16_zfill(void *dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ bool skinny_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag,
                                             const SkinnyParams &p)
 {
@@ -109,11 +129,11 @@ __device__ __forceinline__ void skinny_drain(uint64_t *bar, uint32_t parity, vol
 
 // acc[C0 + j] += v[j] * sa[C0 + j] * sb for j in [0, N): the scale product is
 // rounded once in FP32, then one FMA per element (two per instruction).
-template <int MN, int C0, int N>
-__device__ __forceinline__ void skinny_promote(float (&acc)[MN], const float *v, const float *sa_kb,
+template <int NC, int C0, int N>
+__device__ __forceinline__ void skinny_promote(float (&acc)[NC], const float *v, const float *sa_cols,
                                                float sbv)
 {
-    const float4 *sa4 = reinterpret_cast<const float4 *>(sa_kb + C0);
+    const float4 *sa4 = reinterpret_cast<const float4 *>(sa_cols + C0);
 #pragma unroll
     for (int j = 0; j < N; j += 4) {
         const float4 s = sa4[j / 4]; // same address in every lane: a broadcast
@@ -122,22 +142,28 @@ __device__ __forceinline__ void skinny_promote(float (&acc)[MN], const float *v,
     }
 }
 
-// Promotion of a partial wider than one register batch: chunks of CH columns,
-// each loaded, waited for and multiplied in before the next is loaded.
-template <int MN, int CH, int C = 0>
-__device__ __forceinline__ void skinny_promote_chunks(float (&acc)[MN], float *v, uint32_t taddr,
-                                                      const float *sa_kb, float sbv)
+// The scales of one tile for a CTA's K blocks, as asynchronous copies by one
+// warp: sa[kb][m] for m < M (zero-filled up to MN) and sb[tile][kb].
+template <int MN>
+__device__ __forceinline__ void skinny_copy_scales(const SkinnyParams &p, float *sa_s, float *sb_s,
+                                                   int tile, int kb_lo, int cnt, int lane)
 {
-    if constexpr (C < MN) {
-        tmem_issue_p<CH>(taddr + (uint32_t)C, v);
-        tmem_wait_tie<CH>(v);
-        skinny_promote<MN, C, CH>(acc, v, sa_kb, sbv);
-        skinny_promote_chunks<MN, CH, C + CH>(acc, v, taddr, sa_kb, sbv);
+    constexpr int C4 = MN / 4; // 16-byte chunks per K block
+    for (int idx = lane; idx < cnt * C4; idx += 32) {
+        const int i = idx / C4;
+        const int m = (idx - i * C4) * 4;
+        const int avail = p.M - m;
+        const uint32_t bytes = avail >= 4 ? 16u : (avail > 0 ? 4u * (uint32_t)avail : 0u);
+        // a chunk past M reads nothing (a valid address is still given)
+        const float *src = p.sa + (size_t)(kb_lo + i) * p.ld_sa + (bytes ? m : 0);
+        cp_async_16_zfill(sa_s + i * MN + m, src, bytes);
     }
+    for (int i = lane; i < cnt; i += 32)
+        cp_async_4(sb_s + i, p.sb + (size_t)tile * p.nkb + kb_lo + i);
 }
 
 template <int MN>
-__global__ void __launch_bounds__(SKINNY_THREADS, 1)
+__global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     fp8_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmap_a,
                            const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ SkinnyParams p)
@@ -161,6 +187,7 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
     uint64_t *tmem_empty = done + DONE_RING;
     uint64_t *scales_full = tmem_empty + MAX_TMEM_BUFS;
     uint64_t *mma_done = scales_full + 1;
+    uint64_t *recv_full = mma_done + 1; // split > 1: the tile's slices from every CTA arrived
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + p.off_misc);
     volatile uint32_t *abort_flag = misc + 1;
     float *sa_s = reinterpret_cast<float *>(smem + p.off_sa);
@@ -172,56 +199,87 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
     const int kb_lo = (int)((long)rank * p.nkb / p.split);
     const int kb_hi = (int)((long)(rank + 1) * p.nkb / p.split);
     const int cnt = kb_hi - kb_lo;
-    const uint32_t stage_tx = T::B_BYTES + T::A_BYTES;
     const int t_first = (int)blockIdx.y;
     const int t_stride = (int)gridDim.y;
+    // the output items (one row m, 8 consecutive columns) of a tile that CTA
+    // r of the cluster sums and stores: [r * items / split, (r + 1) * items / split)
+    const int items = p.M * (SKINNY_TILE_N / 8);
+    auto item_lo = [&](int r) { return (int)((long)r * items / p.split); };
+    const uint32_t slot_bytes = skinny_recv_slot_items(p.M, p.split) * 32u;
+    const uint32_t my_bytes = (uint32_t)(item_lo(rank + 1) - item_lo(rank)) * 32u;
 
+    // warp 0 copies B, warp 3 copies A into stage s (each with its bytes)
+    const bool b_side = warp == 0;
     auto issue_load = [&](int s, int kb, int n0) {
         uint8_t *dst = smem + (uint32_t)s * p.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], stage_tx);
-        tma_load_2d(dst, &tmap_b, &full[s], kb * BLOCK_K, n0);
-        tma_load_2d(dst + T::B_BYTES, &tmap_a, &full[s], kb * BLOCK_K, 0);
+        if (b_side) {
+            mbar_arrive_expect_tx(&full[s], T::B_BYTES);
+            tma_load_2d(dst, &tmap_b, &full[s], kb * BLOCK_K, n0);
+        } else {
+            mbar_arrive_expect_tx(&full[s], T::A_BYTES);
+            tma_load_2d(dst + T::B_BYTES, &tmap_a, &full[s], kb * BLOCK_K, 0);
+        }
     };
 
     // ---------------------------------------------------------------- set-up
-    // Thread 0 initialises the barriers and issues the first tile's first
-    // stages at once, before the CTA-wide barrier, so that the copies start as
-    // early as possible; warp 1 allocates TMEM meanwhile.
-    int first = 0;
+    // Thread 0 initialises the stage barriers and issues the first tile's
+    // first stages at once, then the other barriers; warp 1 allocates TMEM and
+    // warp 2 starts the first tile's scale copies meanwhile.  Launched with
+    // programmatic dependent launch, this set-up overlaps the end of the
+    // previous kernel: no thread touches global memory (the operands may be
+    // that kernel's output, D its input) before the dependency wait.
+    const int first = (t_first < p.n_tiles) ? (cnt < stages ? cnt : stages) : 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s)
-            mbar_init(&full[s], 1);
-        for (int j = 0; j < DONE_RING; ++j)
-            mbar_init(&done[j], 1);
-        for (int b = 0; b < T::NBUF; ++b)
-            mbar_init(&tmem_empty[b], 4);
-        mbar_init(scales_full, 32);
-        mbar_init(mma_done, 1);
-        misc[1] = 0u;
+            mbar_init(&full[s], 2);
         fence_mbarrier_init();
         tma_prefetch_desc(&tmap_b);
         tma_prefetch_desc(&tmap_a);
-        if (t_first < p.n_tiles) {
-            first = cnt < stages ? cnt : stages;
-            for (int i = 0; i < first; ++i)
-                issue_load(i, kb_lo + i, t_first * SKINNY_TILE_N);
-        }
     }
     if (warp == 1) {
         tmem_alloc(misc, T::TMEM_COLS);
         tmem_relinquish();
     }
+    grid_dependency_wait();
+    if (warp == 0 || warp == 3) {
+        named_barrier_sync(1, 64); // the stage barriers are initialised
+        if (lane == 0)
+            for (int i = 0; i < first; ++i)
+                issue_load(i, kb_lo + i, t_first * SKINNY_TILE_N);
+    }
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < DONE_RING; ++j)
+            mbar_init(&done[j], 1);
+        for (int b = 0; b < T::NBUF; ++b)
+            mbar_init(&tmem_empty[b], 4 * T::EPI_WGS);
+        mbar_init(scales_full, 32);
+        mbar_init(mma_done, 1);
+        mbar_init(recv_full, 1);
+        // the first tile's slices from the cluster: expected before any can arrive
+        if (p.split > 1 && t_first < p.n_tiles)
+            mbar_arrive_expect_tx(recv_full, (uint32_t)p.split * my_bytes);
+        misc[1] = 0u;
+        fence_mbarrier_init();
+    }
+    if (warp == 2 && t_first < p.n_tiles)
+        skinny_copy_scales<MN>(p, sa_s, sb_s, t_first, kb_lo, cnt, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
+    // the next kernel may start its own set-up on SMs this grid leaves free
+    grid_launch_dependents();
+    // the cluster's barriers are initialised before any CTA sends a slice:
+    // arrive now, wait before the first send
+    if (p.split > 1)
+        cluster_arrive();
 
     uint32_t g0 = 0; // this CTA's K blocks of earlier tiles (ring position)
     int tile_it = 0;
     for (int tile = t_first; tile < p.n_tiles; tile += t_stride, g0 += (uint32_t)cnt, ++tile_it) {
         const int n0 = tile * SKINNY_TILE_N;
-        if (warp == 0) {
-            // -------------------------------------------------------- producer
+        if (warp == 0 || warp == 3) {
+            // -------------------------------------------------------- producers
             if (lane == 0) {
                 uint32_t issued = g0 + (uint32_t)(tile_it == 0 ? first : 0);
                 for (uint32_t g = issued; g < g0 + (uint32_t)cnt; ++g) {
@@ -273,26 +331,21 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
             }
         } else if (warp == 2) {
             // -------------------------------------------------------- scales
-            // LHS scales of rows m < M for the CTA's K blocks (zero for the
-            // padding rows, whose partial columns are zero and never stored),
-            // and the tile's RHS scale per K block.  The previous tile's have
-            // been read (the end-of-tile barriers).
-            for (int idx = lane; idx < cnt * MN; idx += 32) {
-                const int i = idx / MN;
-                const int m = idx - i * MN;
-                sa_s[idx] = m < p.M ? __ldg(p.sa + (size_t)(kb_lo + i) * p.ld_sa + m) : 0.0f;
-            }
-            for (int i = lane; i < cnt; i += 32)
-                sb_s[i] = __ldg(p.sb + (size_t)tile * p.nkb + kb_lo + i);
-            mbar_arrive(scales_full);
+            // the tile's scale copies (the first tile's were started at entry;
+            // the previous tile's have been read: the end-of-tile barriers)
+            if (tile_it > 0)
+                skinny_copy_scales<MN>(p, sa_s, sb_s, tile, kb_lo, cnt, lane);
+            cp_async_mbar_arrive_noinc(scales_full);
         } else if (warp >= 4) {
             // -------------------------------------------------------- epilogue
-            const int q = warp - 4;               // TMEM lane quarter
-            const int row = q * 32 + lane;        // B row within the tile = column of D
-            const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16);
-            float acc[MN];
+            constexpr int NC = T::COLS;
+            const int q = warp & 3;                   // TMEM lane quarter
+            const int col0 = ((warp - 4) >> 2) * NC;  // this warpgroup's columns
+            const int row = q * 32 + lane;            // B row within the tile = column of D
+            const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
+            float acc[NC];
 #pragma unroll
-            for (int j = 0; j < MN; ++j)
+            for (int j = 0; j < NC; ++j)
                 acc[j] = 0.0f;
             bool ok = true;
             auto wait_done = [&](uint32_t g) {
@@ -314,23 +367,23 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
                 if constexpr (T::PREFETCH) {
                     // cur holds K block i (loaded and waited): hand its buffer
                     // back, start loading K block i + 1 into nxt, promote cur
-                    float va[MN], vb[MN];
-                    auto step = [&](float (&cur)[MN], float (&nxt)[MN], int i) {
+                    float va[NC], vb[NC];
+                    auto step = [&](float (&cur)[NC], float (&nxt)[NC], int i) {
                         release(g0 + (uint32_t)i);
                         const bool more = i + 1 < cnt;
                         if (more) {
                             if (!wait_done(g0 + (uint32_t)i + 1))
                                 return false;
-                            tmem_issue_p<MN>(buf_addr(g0 + (uint32_t)i + 1), nxt);
+                            tmem_issue_p<NC>(buf_addr(g0 + (uint32_t)i + 1), nxt);
                         }
-                        skinny_promote<MN, 0, MN>(acc, cur, sa_s + i * MN, sb_s[i]);
+                        skinny_promote<NC, 0, NC>(acc, cur, sa_s + i * MN + col0, sb_s[i]);
                         if (more)
-                            tmem_wait_tie<MN>(nxt);
+                            tmem_wait_tie<NC>(nxt);
                         return true;
                     };
                     if (ok && wait_done(g0)) {
-                        tmem_issue_p<MN>(buf_addr(g0), va);
-                        tmem_wait_tie<MN>(va);
+                        tmem_issue_p<NC>(buf_addr(g0), va);
+                        tmem_wait_tie<NC>(va);
                     } else {
                         ok = false;
                     }
@@ -345,15 +398,23 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
                         }
                     }
                 } else {
-                    float v[T::CHUNK];
+                    // the partial in two halves, each loaded, waited for and
+                    // promoted in turn (registers are fewer at 384 threads)
+                    constexpr int CH = NC / 2;
+                    float v[CH];
                     for (int i = 0; ok && i < cnt; ++i) {
                         const uint32_t g = g0 + (uint32_t)i;
                         if (!wait_done(g)) {
                             ok = false;
                             break;
                         }
-                        skinny_promote_chunks<MN, T::CHUNK>(acc, v, buf_addr(g), sa_s + i * MN, sb_s[i]);
+                        tmem_issue_p<CH>(buf_addr(g), v);
+                        tmem_wait_tie<CH>(v);
+                        skinny_promote<NC, 0, CH>(acc, v, sa_s + i * MN + col0, sb_s[i]);
+                        tmem_issue_p<CH>(buf_addr(g) + (uint32_t)CH, v);
+                        tmem_wait_tie<CH>(v);
                         release(g);
+                        skinny_promote<NC, CH, CH>(acc, v, sa_s + i * MN + col0, sb_s[i]);
                     }
                 }
             }
@@ -364,63 +425,82 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
             if (ok) {
                 float *red = reinterpret_cast<float *>(smem);
 #pragma unroll
-                for (int j = 0; j < MN; ++j)
-                    red[j * SKINNY_TILE_N + row] = acc[j];
+                for (int j = 0; j < NC; ++j)
+                    red[(col0 + j) * SKINNY_TILE_N + row] = acc[j];
+                fence_proxy_async_smem(); // the bulk copies below read it
             }
         }
         __syncwarp();
 
         // ------------------------------------------------------------ reduce + store
-        // Every CTA of the cluster holds its partial tile; CTA r sums a share
-        // of the output items (one row m, 8 consecutive columns) over all
-        // CTAs in rank order and stores them as BF16.
-        if (p.split > 1)
+        __syncthreads(); // the partial tile is complete
+        const uint32_t red_local = smem_addr(smem);
+        const int lo = item_lo(rank), hi = item_lo(rank + 1);
+        if (p.split > 1) {
+            // Send slice r of this CTA's partial tile (items of CTA r) to CTA
+            // r's receive area, slot `rank`; wait for the tile's slices from
+            // every CTA, sum them in rank order, store.  The receive area is
+            // this CTA's own shared memory outside the operand ring, free
+            // since the previous tile's closing cluster barrier.
+            if (tile_it == 0)
+                cluster_wait();
+            if (threadIdx.x == 0) {
+                const uint32_t recv_local = smem_addr(smem + p.off_recv) + (uint32_t)rank * slot_bytes;
+                const uint32_t bar_local = smem_addr(recv_full);
+                for (int r = 0; r < p.split; ++r) {
+                    const int rlo = item_lo(r), rhi = item_lo(r + 1);
+                    if (rhi > rlo)
+                        bulk_copy_to_cluster(map_shared_rank(recv_local, (uint32_t)r),
+                                             red_local + (uint32_t)rlo * 32u, (uint32_t)(rhi - rlo) * 32u,
+                                             map_shared_rank(bar_local, (uint32_t)r));
+                }
+            }
+            const bool got = hi <= lo || skinny_wait(recv_full, (uint32_t)tile_it & 1u, abort_flag, p);
+            const float *recv = reinterpret_cast<const float *>(smem + p.off_recv);
+            for (int it = lo + (int)threadIdx.x; got && it < hi; it += T::THREADS) {
+                const int m = it >> 4;
+                const int c8 = (it & 15) * 8;
+                const int n = n0 + c8;
+                if (n >= p.N)
+                    continue;
+                float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int q = 0; q < p.split; ++q) {
+                    const float *src = recv + (size_t)q * (slot_bytes / 4) + (size_t)(it - lo) * 8;
+                    const float4 a = *reinterpret_cast<const float4 *>(src);
+                    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+                    sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
+                    sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
+                }
+                st_global_v4(p.D + (size_t)m * p.N + n, pack_bf16x2(sum[0], sum[1]),
+                             pack_bf16x2(sum[2], sum[3]), pack_bf16x2(sum[4], sum[5]),
+                             pack_bf16x2(sum[6], sum[7]));
+            }
+            __syncthreads(); // every thread has read the receive area
+            // the next tile's slices are expected before any can be sent
+            if (threadIdx.x == 0 && tile + t_stride < p.n_tiles && hi > lo)
+                mbar_arrive_expect_tx(recv_full, (uint32_t)p.split * my_bytes);
+            // every CTA has received all its slices (so every copy that read
+            // this CTA's partial tile has completed): the rings can be reused
+            // and no CTA leaves while a copy into it is in flight
             cluster_sync();
-        else
-            __syncthreads();
-        {
-            const int items = p.M * (SKINNY_TILE_N / 8);
-            const int lo = (int)((long)rank * items / p.split);
-            const int hi = (int)((long)(rank + 1) * items / p.split);
-            const uint32_t red_local = smem_addr(smem);
-            for (int it = lo + (int)threadIdx.x; it < hi; it += SKINNY_THREADS) {
+        } else {
+            for (int it = lo + (int)threadIdx.x; it < hi; it += T::THREADS) {
                 const int m = it >> 4;
                 const int c8 = (it & 15) * 8;
                 const int n = n0 + c8;
                 if (n >= p.N)
                     continue;
                 const uint32_t off = (uint32_t)(m * SKINNY_TILE_N + c8) * 4u;
-                float sum[8];
-                if (p.split > 1) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        sum[e] = 0.0f;
-                    for (int r = 0; r < p.split; ++r) {
-                        const uint32_t remote = map_shared_rank(red_local + off, (uint32_t)r);
-                        const float4 a = ld_shared_cluster_v4(remote);
-                        const float4 b = ld_shared_cluster_v4(remote + 16);
-                        sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
-                        sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
-                    }
-                } else {
-                    const float4 a = *reinterpret_cast<const float4 *>(smem + off);
-                    const float4 b = *reinterpret_cast<const float4 *>(smem + off + 16);
-                    sum[0] = a.x; sum[1] = a.y; sum[2] = a.z; sum[3] = a.w;
-                    sum[4] = b.x; sum[5] = b.y; sum[6] = b.z; sum[7] = b.w;
-                }
-                st_global_v4(p.D + (size_t)m * p.N + n, pack_bf16x2(sum[0], sum[1]),
-                             pack_bf16x2(sum[2], sum[3]), pack_bf16x2(sum[4], sum[5]),
-                             pack_bf16x2(sum[6], sum[7]));
+                const float4 a = *reinterpret_cast<const float4 *>(smem + off);
+                const float4 b = *reinterpret_cast<const float4 *>(smem + off + 16);
+                st_global_v4(p.D + (size_t)m * p.N + n, pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                             pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
             }
+            __syncthreads(); // the ring is reused by the next tile
         }
-        // no CTA reuses its ring (next tile) or leaves while a peer still
-        // reads its partial tile
-        if (p.split > 1)
-            cluster_sync();
-        else
-            __syncthreads();
     }
-
+    if (p.split > 1 && t_first >= p.n_tiles)
+        cluster_wait(); // pairs the set-up arrival
     if (warp == 1) {
         if (lane == 0) {
             // all MMAs complete before TMEM is released
@@ -431,6 +511,8 @@ __global__ void __launch_bounds__(SKINNY_THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, T::TMEM_COLS);
     }
+    if (warp == 2)
+        cp_async_wait_all(); // no scale copy outlives the CTA
 }
 
 } // namespace fp8nt

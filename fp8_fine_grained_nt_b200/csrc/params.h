@@ -123,7 +123,6 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
 // D^T tiles: 128 rows of B per tile on the MMA's M side and the rows of A,
 // zero-padded to MN, on its N side (kernel_skinny.cuh).
 
-constexpr int SKINNY_THREADS = 256;      // warps 0-3: roles, warps 4-7: epilogue
 constexpr int SKINNY_TILE_N = 128;       // rows of B (columns of D) per tile
 constexpr int SKINNY_MAX_SPLIT = 8;      // CTAs per cluster sharing a tile's K range
 constexpr int SKINNY_MAX_M = 128;
@@ -139,6 +138,7 @@ struct SkinnyParams {
     int stages;     // operand ring depth
     uint32_t stage_bytes; // 128 x 128 B of B, then MN x 128 B of A
     uint32_t region;      // operand ring, reused for the FP32 partial tile at the end
+    uint32_t off_recv;    // split > 1: the output slices the cluster's CTAs send to this one
     uint32_t off_sa;      // LHS scales of the CTA's K range: kb_max x MN FP32
     uint32_t off_sb;      // RHS scales of the tile's 128-row block: kb_max FP32
     uint32_t off_bars;
@@ -153,17 +153,30 @@ struct SkinnyParams {
 };
 
 // Barriers of the skinny kernel: full per stage, "K block done" ring, TMEM
-// buffer released (ring), scales loaded, all MMAs done.
-constexpr int SKINNY_NUM_BARS_FIXED = DONE_RING + MAX_TMEM_BUFS + 2;
+// buffer released (ring), scales loaded, all MMAs done, partial slices
+// received.
+constexpr int SKINNY_NUM_BARS_FIXED = DONE_RING + MAX_TMEM_BUFS + 3;
+
+// Bytes of the partial tile ([MN][128] FP32) and of the receive area for the
+// slices of the output that the cluster's CTAs send to one CTA: split slots
+// of ceil(items / split) items, an item being 8 FP32 values (items = 16 M).
+__host__ __device__ inline uint32_t skinny_red_bytes(int mn) { return (uint32_t)mn * SKINNY_TILE_N * 4u; }
+__host__ __device__ inline uint32_t skinny_recv_slot_items(int m, int split)
+{
+    const uint32_t items = (uint32_t)m * (SKINNY_TILE_N / 8);
+    return (items + (uint32_t)split - 1) / (uint32_t)split;
+}
 
 __host__ __device__ inline void make_skinny_plan(SkinnyParams &p, int mn, int stages)
 {
     p.stages = stages;
     p.stage_bytes = (uint32_t)(SKINNY_TILE_N + mn) * BLOCK_K;
     const uint32_t ring = p.stage_bytes * (uint32_t)stages;
-    const uint32_t red = (uint32_t)mn * SKINNY_TILE_N * 4u;
+    const uint32_t red = skinny_red_bytes(mn);
     p.region = ring > red ? ring : red;
-    p.off_sa = align_up_u32(p.region, 128);
+    p.off_recv = align_up_u32(p.region, 1024);
+    const uint32_t recv = p.split > 1 ? (uint32_t)p.split * skinny_recv_slot_items(p.M, p.split) * 32u : 0u;
+    p.off_sa = align_up_u32(p.off_recv + recv, 128);
     p.off_sb = p.off_sa + (uint32_t)p.kb_max * (uint32_t)mn * 4u;
     p.off_bars = align_up_u32(p.off_sb + (uint32_t)p.kb_max * 4u, 8);
     p.off_misc = align_up_u32(p.off_bars + 8u * (uint32_t)(stages + SKINNY_NUM_BARS_FIXED), 16);

@@ -59,6 +59,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return done != 0;
 }
 
+// ---------------------------------------------------------------- launch order
+
+// Wait until the grids this one depends on (programmatic dependent launch)
+// have completed and their memory operations are visible; returns at once
+// when there are none.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the grid launched after this one (with programmatic dependent launch)
+// to be scheduled once every CTA of this grid has done so or exited.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
@@ -366,6 +383,38 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr)
                  : "r"(addr)
                  : "memory");
     return v;
+}
+
+// CTA named barrier `id` (1..15) over `count` threads (whole warps).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Split cluster barrier: every thread of every CTA arrives (release: its
+// earlier shared-memory writes and barrier initialisations become visible to
+// the cluster) and later waits (acquire) for all arrivals.
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to a
+// cluster address (another CTA's shared memory, or this one's), completing
+// as transaction bytes on the mbarrier at cluster address `bar_cluster` (in
+// the destination CTA).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                     uint32_t bar_cluster)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- CTA pairs
