@@ -5,12 +5,19 @@
 // the GEMM; the 1x128 granularity is the DeepSeek-V3 recipe.
 //
 // Per block: amax = max |x| (exact), s = max(amax, 1e-4) / 448 and
-// q = E4M3(clamp(x / s, +-448)), both divisions IEEE round-to-nearest, the
-// cast round-to-nearest-even.  HBM-bound: one warp per 32 rows x 128
-// columns, each lane 16 bytes (FP32) or 8 bytes (BF16) of a row at a time,
-// the next four rows' loads in flight while four rows are quantised;
-// lane i keeps row i's scale, so the 32 scales of a block column go out as
-// one coalesced 128-byte store.
+// q = E4M3(clamp(x / s, +-448)), both divisions rounded to nearest (IEEE),
+// the cast round-to-nearest-even.  The per-element quotient x / s comes from
+// the block's correctly rounded reciprocal r = 1/s and one FMA correction
+// step (Markstein's method: q0 = x * r, e = x - q0 * s exactly by FMA,
+// q = q0 + e * r), which yields the correctly rounded quotient when r is the
+// correctly rounded reciprocal, at three operations per element instead of a
+// full division.
+//
+// HBM-bound: one warp per 32 rows x 128 columns, 8 lanes per row, each lane
+// 16 consecutive elements (64 bytes of FP32 or 32 of BF16) of a row; four
+// rows per step with the next step's loads in flight; the amax of a row is
+// three shuffles within its 8 lanes; each lane ends up with the scale of one
+// of the 32 rows, so a block column of scales is one coalesced 128-byte store.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -22,7 +29,6 @@ namespace fp8nt {
 namespace {
 
 constexpr int QUANT_WARPS = 8; // warps per CTA
-constexpr int QUANT_ROWS_IN_FLIGHT = 4;
 
 // Two FP32 values -> two E4M3 bytes (round to nearest even, saturating),
 // low byte = lo.
@@ -33,24 +39,45 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
     return r;
 }
 
+// 16 consecutive elements of a row as FP32.
 template <bool BF16_IN>
-__device__ __forceinline__ void load4(const void *x, long off, float (&v)[4])
+__device__ __forceinline__ void load16(const void *x, long off, float (&v)[16])
 {
     if constexpr (BF16_IN) {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(x) + off));
-        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-        v[0] = __low2float(lo);
-        v[1] = __high2float(lo);
-        v[2] = __low2float(hi);
-        v[3] = __high2float(hi);
+        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + off);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 raw = __ldg(p + h);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                // a BF16 value is the high half of the FP32 with the same bits
+                v[h * 8 + 2 * i] = __uint_as_float(w[i] << 16);
+                v[h * 8 + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            }
+        }
     } else {
-        const float4 f = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(x) + off));
-        v[0] = f.x;
-        v[1] = f.y;
-        v[2] = f.z;
-        v[3] = f.w;
+        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + off);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float4 f = __ldg(p + h);
+            v[4 * h] = f.x;
+            v[4 * h + 1] = f.y;
+            v[4 * h + 2] = f.z;
+            v[4 * h + 3] = f.w;
+        }
     }
+}
+
+// x / s rounded to nearest, given r = 1/s rounded to nearest: one FMA
+// correction of the product x * r (Markstein's method).  A zero residual
+// means q0 is exact; returning it keeps the sign of a zero quotient (-0 / s
+// is -0, which the correction q0 + 0 * r would turn into +0).
+__device__ __forceinline__ float div_by_scale(float x, float s, float r)
+{
+    const float q0 = x * r;
+    const float e = fmaf(-q0, s, x);
+    return e == 0.0f ? q0 : fmaf(e, r, q0);
 }
 
 template <bool BF16_IN>
@@ -66,46 +93,51 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32)
     // consecutive warps take consecutive K blocks of the same 32 rows
     const int kb = (int)(wid % nkb);
     const int r0 = (int)(wid / nkb) * 32;
-    const long col = (long)kb * 128 + lane * 4;
+    const int sub = lane >> 3;                      // row within a step of 4
+    const long col = (long)kb * 128 + (lane & 7) * 16;
     float my_scale = 0.0f;
-    // software pipeline: the next rows' loads are in flight while the
-    // current rows are reduced, divided and stored
-    float v[2][QUANT_ROWS_IN_FLIGHT][4];
-    auto load_rows = [&](int i, float (&dst)[QUANT_ROWS_IN_FLIGHT][4]) {
+    float v[2][16];
+    auto load_step = [&](int it, float (&dst)[16]) {
+        const int row = r0 + it * 4 + sub;
+        if (row < M)
+            load16<BF16_IN>(x, (long)row * K + col, dst);
+        else
 #pragma unroll
-        for (int j = 0; j < QUANT_ROWS_IN_FLIGHT; ++j) {
-            const int row = r0 + i + j;
-            if (row < M)
-                load4<BF16_IN>(x, (long)row * K + col, dst[j]);
-            else
-                dst[j][0] = dst[j][1] = dst[j][2] = dst[j][3] = 0.0f;
-        }
+            for (int e = 0; e < 16; ++e)
+                dst[e] = 0.0f;
     };
-    load_rows(0, v[0]);
+    load_step(0, v[0]);
 #pragma unroll
-    for (int i = 0; i < 32; i += QUANT_ROWS_IN_FLIGHT) {
-        const int cur = (i / QUANT_ROWS_IN_FLIGHT) & 1;
-        if (i + QUANT_ROWS_IN_FLIGHT < 32)
-            load_rows(i + QUANT_ROWS_IN_FLIGHT, v[cur ^ 1]);
+    for (int it = 0; it < 8; ++it) {
+        float(&w)[16] = v[it & 1];
+        if (it + 1 < 8)
+            load_step(it + 1, v[(it + 1) & 1]);
+        float amax = 0.0f;
 #pragma unroll
-        for (int j = 0; j < QUANT_ROWS_IN_FLIGHT; ++j) {
-            const float(&w)[4] = v[cur][j];
-            float amax = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+        for (int e = 0; e < 16; ++e)
+            amax = fmaxf(amax, fabsf(w[e]));
 #pragma unroll
-            for (int d = 16; d > 0; d >>= 1)
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-            const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+        for (int d = 4; d > 0; d >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+        const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+        const float r = __frcp_rn(s);
+        uint32_t packed[4];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
             float y[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                y[e] = fminf(fmaxf(__fdiv_rn(w[e], s), -448.0f), 448.0f);
-            const uint32_t packed = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
-            const int row = r0 + i + j;
-            if (row < M)
-                *reinterpret_cast<uint32_t *>(q + (long)row * K + col) = packed;
-            if (lane == i + j)
-                my_scale = s;
+            for (int i = 0; i < 4; ++i)
+                y[i] = fminf(fmaxf(div_by_scale(w[e + i], s, r), -448.0f), 448.0f);
+            packed[e / 4] = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
         }
+        const int row = r0 + it * 4 + sub;
+        if (row < M)
+            *reinterpret_cast<uint4 *>(q + (long)row * K + col) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        // lane j keeps the scale of row j (rows it * 4 .. it * 4 + 3 now)
+        const float sv = __shfl_sync(0xffffffffu, s, (lane & 3) * 8);
+        if ((lane >> 2) == it)
+            my_scale = sv;
     }
     if (r0 + lane < M)
         sa[(long)kb * ld_sa + r0 + lane] = my_scale;
