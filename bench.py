@@ -46,6 +46,7 @@ from fp8_fine_grained_nt_b200 import inputs  # noqa: E402
 METRIC = "FP8 TFLOPS and % of B200 roofline per shape (dense, contiguous, masked)"
 UNIT = "TFLOP/s"
 NOMINAL_FP8_TFLOPS = 4500.0
+NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 WORKLOAD_NAMES = [
@@ -684,6 +685,10 @@ def run_gpu(args):
             "per_shape": per_shape,
             "roofline": {"kernel": dom.name, "bound": bound, "achieved": round(achieved, 2),
                          "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+                         # the same against the nominal dense FP8 peak (4.5 PFLOP/s)
+                         # or the nominal 8 TB/s HBM, for comparison
+                         "frac_of_nominal": round(achieved / (NOMINAL_FP8_TFLOPS if bound == "tensor"
+                                                              else NOMINAL_HBM_GBS), 4),
                          "traffic": traffic,
                          "peak_source": (f"{peaks['source']}: "
                                          + ("2 x bf16 burst (fp8:bf16 nominal ratio 2)"

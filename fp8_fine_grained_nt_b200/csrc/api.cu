@@ -448,9 +448,10 @@ int cluster_capacity_model(int split, int sms)
 // its share of K blocks at the slowest of (a) the four MMAs of a K block (at
 // least ~64 cycles each for one issuing thread, ~75 at N = 128), (b) its share
 // of the HBM bandwidth (~3300 B/clk at the boost clock) for 16 KB of B per K
-// block, (c) one SM's TMA ingest (~110 B/clk); plus set-up and, with a
-// cluster, the reduction of the partial tiles through distributed shared
-// memory.
+// block, (c) what one CTA's operand ring keeps in flight: measured on B200
+// (decode shape, 34 to 102 CTAs) a CTA takes in ~30 B/clk whatever the
+// number of CTAs, so more CTAs stream faster until (b) binds; plus set-up
+// and, with a cluster, the exchange of the partial tiles.
 double skinny_cycles(int N, int K, int mn, int split, int cap)
 {
     const long tiles = ceil_div(N, SKINNY_TILE_N);
@@ -460,7 +461,7 @@ double skinny_cycles(int N, int K, int mn, int split, int cap)
     const int cnt = ceil_div(nkb, split);
     const double t_mma = 4.0 * (mn <= 64 ? 64.0 : 75.0);
     const double t_hbm = 128.0 * 128.0 * (double)active / 3300.0;
-    const double t_tma = (128.0 + mn) * 128.0 / 110.0;
+    const double t_tma = (128.0 + mn) * 128.0 / 30.0;
     double t_kb = t_mma > t_hbm ? t_mma : t_hbm;
     t_kb = t_kb > t_tma ? t_kb : t_tma;
     return (double)waves * (1200.0 + cnt * t_kb + (split > 1 ? 800.0 + 100.0 * split : 300.0));
@@ -485,14 +486,19 @@ bool skinny_plan(const Problem &pb, int mn, int split, int max_smem, SkinnyParam
     p.nkb = pb.K / 128;
     p.n_tiles = ceil_div(pb.N, SKINNY_TILE_N);
     p.split = split;
-    p.kb_max = ceil_div(p.nkb, split);
-    int st = p.kb_max < DONE_RING ? p.kb_max : DONE_RING;
+    const int units = ceil_div(p.nkb, SKINNY_KB_PER_STAGE);
+    const int unit_max = ceil_div(units, split);
+    p.kb_max = unit_max * SKINNY_KB_PER_STAGE;
+    // stages (each KB_PER_STAGE K blocks) in flight stay within the ring of
+    // "K block done" barriers
+    const int st_cap = DONE_RING / SKINNY_KB_PER_STAGE;
+    int st = unit_max < st_cap ? unit_max : st_cap;
     for (; st >= 1; --st) {
         make_skinny_plan(p, mn, st);
         if ((int)p.total + 1024 <= max_smem)
             break;
     }
-    if (st < 1 || (st < 2 && p.kb_max > 1))
+    if (st < 1 || (st < 2 && unit_max > 1))
         return false;
     *out = p;
     return true;
@@ -625,14 +631,27 @@ int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const void *A, const
     if (st != DG_OK)
         return st;
     CUtensorMap tmap_a, tmap_b;
-    // A: [M][K] bytes, box MN rows x 128 (rows past M are zero-filled); B:
-    // [N][K] bytes, box 128 rows x 128
+    // A: [M][K] bytes, box MN rows x 128 (rows past M are zero-filled)
     if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, pb.M, pb.K, 128,
                            (uint32_t)ch.cand->mn, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
         return st;
-    if ((st = make_tmap_2d(&tmap_b, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, pb.N, pb.K, 128,
-                           SKINNY_TILE_N, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK)
-        return st;
+    // B: [N][K] bytes viewed in 4-D as [N/8 row groups][K/128 K blocks][8 rows]
+    // [128 bytes] (N % 8 == 0), box = 16 row groups x KB_PER_STAGE K blocks:
+    // the tile's 128 rows of KB_PER_STAGE consecutive K blocks, laid out in
+    // shared memory as [row group][K block][8 rows][128 B] (128-byte swizzle)
+    {
+        EncodeTiledFn fn = encode_fn();
+        if (!fn)
+            return DG_ERR_CUDA;
+        cuuint64_t dims[4] = {128, 8, (cuuint64_t)(pb.K / 128), (cuuint64_t)(pb.N / 8)};
+        cuuint64_t strides[3] = {(cuuint64_t)pb.K, 128, (cuuint64_t)pb.K * 8};
+        cuuint32_t box[4] = {128, 8, SKINNY_KB_PER_STAGE, SKINNY_TILE_N / 8};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (fn(&tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(B), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return DG_ERR_CUDA;
+    }
     SkinnyParams p = ch.plan;
     p.sa = sa;
     p.ld_sa = get_tma_aligned_size(pb.M, 4);

@@ -103,6 +103,13 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr)
            | ((uint64_t)2u << 61);              // layout: 128-byte swizzle
 }
 
+// The same with a given stride between 8-row groups (bytes, a multiple of 16).
+__device__ __forceinline__ uint64_t make_sdesc_sbo(uint32_t saddr, uint32_t sbo_bytes)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
 struct TileInfo {
     int valid;   // 0: nothing to compute (contiguous padding block, bad expert)
     int g;       // group (masked) / expert (contiguous) / 0 (dense)

@@ -193,12 +193,16 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     float *sa_s = reinterpret_cast<float *>(smem + p.off_sa);
     float *sb_s = reinterpret_cast<float *>(smem + p.off_sb);
 
-    // a cluster of `split` CTAs works on one tile at a time, CTA r on K blocks
-    // [r * nkb / split, (r + 1) * nkb / split); clusters stride over the tiles
+    // a cluster of `split` CTAs works on one tile at a time, CTA r on the K
+    // blocks of stages [r * units / split, (r + 1) * units / split), a stage
+    // being G = SKINNY_KB_PER_STAGE K blocks; clusters stride over the tiles
+    constexpr int G = SKINNY_KB_PER_STAGE;
     const int rank = p.split > 1 ? (int)cluster_ctarank() : 0;
-    const int kb_lo = (int)((long)rank * p.nkb / p.split);
-    const int kb_hi = (int)((long)(rank + 1) * p.nkb / p.split);
-    const int cnt = kb_hi - kb_lo;
+    const int units = (p.nkb + G - 1) / G;
+    const int kb_lo = G * (int)((long)rank * units / p.split);
+    const int kb_hi = min(p.nkb, G * (int)((long)(rank + 1) * units / p.split));
+    const int cnt = max(0, kb_hi - kb_lo);
+    const int ucnt = (cnt + G - 1) / G; // stages per tile
     const int t_first = (int)blockIdx.y;
     const int t_stride = (int)gridDim.y;
     // the output items (one row m, 8 consecutive columns) of a tile that CTA
@@ -208,17 +212,26 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     const uint32_t slot_bytes = skinny_recv_slot_items(p.M, p.split) * 32u;
     const uint32_t my_bytes = (uint32_t)(item_lo(rank + 1) - item_lo(rank)) * 32u;
 
-    // warp 0 copies B, warp 3 copies A into stage s (each with its bytes)
+    // warp 0 copies B, warp 3 copies A into stage s (each with its bytes):
+    // K blocks [kb, kb + G) (any past K are zero-filled and not used)
     const bool b_side = warp == 0;
     auto issue_load = [&](int s, int kb, int n0) {
         uint8_t *dst = smem + (uint32_t)s * p.stage_bytes;
         if (b_side) {
-            mbar_arrive_expect_tx(&full[s], T::B_BYTES);
-            tma_load_2d(dst, &tmap_b, &full[s], kb * BLOCK_K, n0);
+            mbar_arrive_expect_tx(&full[s], G * T::B_BYTES);
+            tma_load_4d(dst, &tmap_b, &full[s], 0, 0, kb, n0 / 8);
         } else {
-            mbar_arrive_expect_tx(&full[s], T::A_BYTES);
-            tma_load_2d(dst + T::B_BYTES, &tmap_a, &full[s], kb * BLOCK_K, 0);
+            mbar_arrive_expect_tx(&full[s], G * T::A_BYTES);
+#pragma unroll
+            for (int z = 0; z < G; ++z)
+                tma_load_2d(dst + G * T::B_BYTES + z * T::A_BYTES, &tmap_a, &full[s], (kb + z) * BLOCK_K, 0);
         }
+    };
+    // the last K block (counted over this CTA's tiles) that stage use u holds
+    auto last_kb_of_use = [&](uint32_t u) {
+        const uint32_t t = u / (uint32_t)ucnt, j = u % (uint32_t)ucnt;
+        const uint32_t end = (j + 1) * G < (uint32_t)cnt ? (j + 1) * G : (uint32_t)cnt;
+        return t * (uint32_t)cnt + end - 1;
     };
 
     // ---------------------------------------------------------------- set-up
@@ -228,7 +241,7 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     // programmatic dependent launch, this set-up overlaps the end of the
     // previous kernel: no thread touches global memory (the operands may be
     // that kernel's output, D its input) before the dependency wait.
-    const int first = (t_first < p.n_tiles) ? (cnt < stages ? cnt : stages) : 0;
+    const int first = (t_first < p.n_tiles) ? (ucnt < stages ? ucnt : stages) : 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s)
             mbar_init(&full[s], 2);
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
         named_barrier_sync(1, 64); // the stage barriers are initialised
         if (lane == 0)
             for (int i = 0; i < first; ++i)
-                issue_load(i, kb_lo + i, t_first * SKINNY_TILE_N);
+                issue_load(i, kb_lo + G * i, t_first * SKINNY_TILE_N);
     }
     if (threadIdx.x == 0) {
         for (int j = 0; j < DONE_RING; ++j)
@@ -270,63 +283,77 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     // the next kernel may start its own set-up on SMs this grid leaves free
     grid_launch_dependents();
     // the cluster's barriers are initialised before any CTA sends a slice:
-    // arrive now, wait before the first send
+    // arrive now, wait before the first send (the initialisation is ordered
+    // by fence.mbarrier_init; a releasing arrive would also wait for this
+    // thread's earlier memory operations)
     if (p.split > 1)
-        cluster_arrive();
+        cluster_arrive_relaxed();
 
     uint32_t g0 = 0; // this CTA's K blocks of earlier tiles (ring position)
+    uint32_t u0 = 0; // this CTA's stage uses of earlier tiles
     int tile_it = 0;
-    for (int tile = t_first; tile < p.n_tiles; tile += t_stride, g0 += (uint32_t)cnt, ++tile_it) {
+    for (int tile = t_first; tile < p.n_tiles;
+         tile += t_stride, g0 += (uint32_t)cnt, u0 += (uint32_t)ucnt, ++tile_it) {
         const int n0 = tile * SKINNY_TILE_N;
         if (warp == 0 || warp == 3) {
             // -------------------------------------------------------- producers
             if (lane == 0) {
-                uint32_t issued = g0 + (uint32_t)(tile_it == 0 ? first : 0);
-                for (uint32_t g = issued; g < g0 + (uint32_t)cnt; ++g) {
-                    const int s = (int)(g % (uint32_t)stages);
-                    if (g >= (uint32_t)stages) {
-                        // stage s was last used by K block g - stages
-                        const uint32_t j = g - (uint32_t)stages;
+                uint32_t issued = u0 + (uint32_t)(tile_it == 0 ? first : 0);
+                for (uint32_t u = issued; u < u0 + (uint32_t)ucnt; ++u) {
+                    const int s = (int)(u % (uint32_t)stages);
+                    if (u >= (uint32_t)stages) {
+                        // stage s was last used by stage use u - stages:
+                        // free once its last K block's MMAs completed
+                        const uint32_t j = last_kb_of_use(u - (uint32_t)stages);
                         if (!skinny_wait(&done[j % DONE_RING], (j / DONE_RING) & 1u, abort_flag, p))
                             break;
                     }
-                    issue_load(s, kb_lo + (int)(g - g0), n0);
-                    issued = g + 1;
+                    issue_load(s, kb_lo + G * (int)(u - u0), n0);
+                    issued = u + 1;
                 }
                 // every copy issued must land before the ring is reused for
                 // the partial tile or the CTA exits (normally the MMAs have
                 // consumed them all)
                 const uint32_t n = issued < (uint32_t)stages ? issued : (uint32_t)stages;
-                for (uint32_t g = issued - n; g < issued; ++g)
-                    skinny_drain(&full[g % stages], (g / stages) & 1u, abort_flag, p);
+                for (uint32_t u = issued - n; u < issued; ++u)
+                    skinny_drain(&full[u % stages], (u / stages) & 1u, abort_flag, p);
             }
         } else if (warp == 1) {
             // -------------------------------------------------------- MMA issuer
             if (lane == 0) {
                 // D^T tile: the B tile is the MMA's A operand (M = 128), the A
                 // tile its B operand (N = MN); both K-major, 128-byte swizzle.
+                // K block z of a stage: B's 8-row groups are G KB apart
+                // ([row group][K block][8 rows][128 B]), A's tile is whole.
                 constexpr uint32_t idesc = make_idesc(MN, SKINNY_TILE_N);
-                const uint64_t a_desc0 = make_sdesc(smem_addr(smem));
-                const uint64_t b_desc0 = make_sdesc(smem_addr(smem) + T::B_BYTES);
+                const uint64_t a_desc0 = make_sdesc_sbo(smem_addr(smem), G * 1024u);
+                const uint64_t b_desc0 = make_sdesc(smem_addr(smem) + G * T::B_BYTES);
                 const uint32_t stage_step = p.stage_bytes >> 4;
-                for (uint32_t g = g0; g < g0 + (uint32_t)cnt; ++g) {
-                    const uint32_t s = g % (uint32_t)stages;
-                    if (!skinny_wait(&full[s], (g / (uint32_t)stages) & 1u, abort_flag, p))
+                uint32_t g = g0;
+                bool ok = true;
+                for (uint32_t u = u0; ok && u < u0 + (uint32_t)ucnt; ++u) {
+                    const uint32_t s = u % (uint32_t)stages;
+                    if (!skinny_wait(&full[s], (u / (uint32_t)stages) & 1u, abort_flag, p))
                         break;
-                    const uint32_t buf = g % T::NBUF;
-                    if (g >= (uint32_t)T::NBUF &&
-                        !skinny_wait(&tmem_empty[buf], (g / T::NBUF - 1) & 1u, abort_flag, p))
-                        break;
-                    tc_fence_after();
-                    const uint32_t d = tmem_base + buf * (uint32_t)MN;
-                    const uint64_t ad = a_desc0 + (uint64_t)(s * stage_step);
-                    const uint64_t bd = b_desc0 + (uint64_t)(s * stage_step);
+                    const int kbs = min(G, cnt - G * (int)(u - u0)); // K blocks of this stage
+                    for (int z = 0; z < kbs; ++z, ++g) {
+                        const uint32_t buf = g % T::NBUF;
+                        if (g >= (uint32_t)T::NBUF &&
+                            !skinny_wait(&tmem_empty[buf], (g / T::NBUF - 1) & 1u, abort_flag, p)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d = tmem_base + buf * (uint32_t)MN;
+                        const uint64_t ad = a_desc0 + (uint64_t)(s * stage_step + ((uint32_t)z * 1024u >> 4));
+                        const uint64_t bd = b_desc0 + (uint64_t)(s * stage_step + ((uint32_t)z * T::A_BYTES >> 4));
 #pragma unroll
-                    for (int k = 0; k < BLOCK_K / MMA_K; ++k)
-                        mma_f8f6f4(d, ad + (uint64_t)((k * MMA_K) >> 4), bd + (uint64_t)((k * MMA_K) >> 4),
-                                   idesc, k > 0 ? 1u : 0u);
-                    // frees the stage and publishes the partial
-                    mma_commit(&done[g % DONE_RING]);
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
+                            mma_f8f6f4(d, ad + (uint64_t)((k * MMA_K) >> 4), bd + (uint64_t)((k * MMA_K) >> 4),
+                                       idesc, k > 0 ? 1u : 0u);
+                        // publishes the partial (the stage's last one also frees it)
+                        mma_commit(&done[g % DONE_RING]);
+                    }
                 }
             }
         } else if (warp == 2) {
@@ -444,16 +471,15 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
             // since the previous tile's closing cluster barrier.
             if (tile_it == 0)
                 cluster_wait();
-            if (threadIdx.x == 0) {
+            if (threadIdx.x < p.split) {
+                // lane r of warp 0 sends slice r (the copies are issued in parallel)
+                const int r = (int)threadIdx.x;
+                const int rlo = item_lo(r), rhi = item_lo(r + 1);
                 const uint32_t recv_local = smem_addr(smem + p.off_recv) + (uint32_t)rank * slot_bytes;
-                const uint32_t bar_local = smem_addr(recv_full);
-                for (int r = 0; r < p.split; ++r) {
-                    const int rlo = item_lo(r), rhi = item_lo(r + 1);
-                    if (rhi > rlo)
-                        bulk_copy_to_cluster(map_shared_rank(recv_local, (uint32_t)r),
-                                             red_local + (uint32_t)rlo * 32u, (uint32_t)(rhi - rlo) * 32u,
-                                             map_shared_rank(bar_local, (uint32_t)r));
-                }
+                if (rhi > rlo)
+                    bulk_copy_to_cluster(map_shared_rank(recv_local, (uint32_t)r),
+                                         red_local + (uint32_t)rlo * 32u, (uint32_t)(rhi - rlo) * 32u,
+                                         map_shared_rank(smem_addr(recv_full), (uint32_t)r));
             }
             const bool got = hi <= lo || skinny_wait(recv_full, (uint32_t)tile_it & 1u, abort_flag, p);
             const float *recv = reinterpret_cast<const float *>(smem + p.off_recv);

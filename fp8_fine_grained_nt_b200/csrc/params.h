@@ -126,6 +126,10 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
 constexpr int SKINNY_TILE_N = 128;       // rows of B (columns of D) per tile
 constexpr int SKINNY_MAX_SPLIT = 8;      // CTAs per cluster sharing a tile's K range
 constexpr int SKINNY_MAX_M = 128;
+// K blocks per operand stage: B arrives as one 4-D box holding these K blocks
+// of each 8-row group, so every row's KB_PER_STAGE * 128 bytes are fetched
+// together (longer contiguous reads from HBM than one K block at a time)
+constexpr int SKINNY_KB_PER_STAGE = 2;
 
 struct SkinnyParams {
     int M;          // rows of A and D (<= MN of the kernel)
@@ -134,9 +138,11 @@ struct SkinnyParams {
     int nkb;        // K / 128
     int n_tiles;    // ceil(N / 128)
     int split;      // CTAs of a cluster that share one tile, each a contiguous K range
-    int kb_max;     // K blocks of the largest share: ceil(nkb / split)
-    int stages;     // operand ring depth
-    uint32_t stage_bytes; // 128 x 128 B of B, then MN x 128 B of A
+                    // (whole stages of SKINNY_KB_PER_STAGE K blocks)
+    int kb_max;     // K blocks of the largest share
+    int stages;     // operand ring depth (each stage SKINNY_KB_PER_STAGE K blocks)
+    uint32_t stage_bytes; // B: [16 row groups][KB_PER_STAGE][8 rows][128 B]; then A:
+                          // [KB_PER_STAGE][MN rows][128 B]
     uint32_t region;      // operand ring, reused for the FP32 partial tile at the end
     uint32_t off_recv;    // split > 1: the output slices the cluster's CTAs send to this one
     uint32_t off_sa;      // LHS scales of the CTA's K range: kb_max x MN FP32
@@ -170,7 +176,7 @@ __host__ __device__ inline uint32_t skinny_recv_slot_items(int m, int split)
 __host__ __device__ inline void make_skinny_plan(SkinnyParams &p, int mn, int stages)
 {
     p.stages = stages;
-    p.stage_bytes = (uint32_t)(SKINNY_TILE_N + mn) * BLOCK_K;
+    p.stage_bytes = (uint32_t)SKINNY_KB_PER_STAGE * (SKINNY_TILE_N + mn) * BLOCK_K;
     const uint32_t ring = p.stage_bytes * (uint32_t)stages;
     const uint32_t red = skinny_red_bytes(mn);
     p.region = ring > red ? ring : red;

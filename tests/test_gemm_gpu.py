@@ -304,10 +304,23 @@ def test_full_size_contiguous():
             edge_rows += [s, last]
     rows = np.concatenate([rows, np.repeat(edge_rows, prob.N)])
     cols = np.concatenate([cols, np.tile(np.arange(prob.N), len(edge_rows))])
+    # one whole 128 x 256 output tile at an expert boundary: the last, partly
+    # padded M block of the first expert whose count is not a multiple of 128,
+    # every row of it (valid rows compared, padding rows must keep the sentinel)
+    # over the tile's 256 columns at the end of N
+    e_b = next(e for e, c in enumerate(prob.counts) if c % 128 != 0)
+    seg0 = sum(-(-c // 128) * 128 for c in prob.counts[:e_b])
+    blk0 = seg0 + (prob.counts[e_b] // 128) * 128
+    t_rows = np.arange(blk0, blk0 + 128)
+    t_valid = t_rows[mi[t_rows] >= 0]
+    t_cols = np.arange(prob.N - 256, prob.N)
+    rows = np.concatenate([rows, np.repeat(t_valid, 256)])
+    cols = np.concatenate([cols, np.tile(t_cols, len(t_valid))])
     ref = oracle.gemm_contiguous_sampled(prob.a, prob.sa, prob.b, prob.sb, prob.m_indices,
                                          prob.num_groups, prob.M_sum, prob.N, prob.K, rows, cols)
     H.assert_close(got[rows, cols], ref, "contiguous full")
     assert H.untouched(d)[mi < 0].all(), "padding rows were written"
+    assert 0 < len(t_valid) < 128 and H.untouched(d)[t_rows[mi[t_rows] < 0]][:, t_cols].all()
 
 
 @pytest.mark.parametrize("name", ["masked_16x256_4096x7168", "masked_16x256_7168x2048"])
