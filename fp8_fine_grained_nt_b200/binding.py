@@ -35,6 +35,7 @@ __all__ = [
     "select_config",
     "force_config",
     "force_swap_ab",
+    "force_tail_split",
     "status_string",
     "KIND_DENSE",
     "KIND_CONTIGUOUS",
@@ -62,7 +63,7 @@ class DgConfig(ctypes.Structure):
                 ("num_tiles", ctypes.c_int), ("grid", ctypes.c_int),
                 ("smem_bytes", ctypes.c_int), ("tmem_cols", ctypes.c_int),
                 ("split", ctypes.c_int), ("cta_pair", ctypes.c_int),
-                ("swap_ab", ctypes.c_int)]
+                ("swap_ab", ctypes.c_int), ("tail_tiles", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -100,6 +101,7 @@ def load_library():
         lib.dg_select_config.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(DgConfig)]
         lib.dg_force_config.argtypes = [I, I, I, I]
         lib.dg_force_swap_ab.argtypes = [I]
+        lib.dg_force_tail_split.argtypes = [I]
         _lib = lib
         return lib
 
@@ -301,6 +303,13 @@ def force_config(block_m: int = 0, block_n: int = 0, split: int = 0, cta_pair: i
 
 
 def force_swap_ab(mode: int = 0) -> None:
-    """Small-M kernel choice for later dense calls: 0 = automatic (M <= 128
+    """Small-M kernel choice for later dense calls: 0 = automatic (M <= 256
     uses it), 1 = never, 2 = wherever it applies.  For tests."""
     _check(load_library().dg_force_swap_ab(int(mode)), "dg_force_swap_ab")
+
+
+def force_tail_split(mode: int = 0) -> None:
+    """Split of a dense call's last partial wave onto the small-M kernel:
+    0 = automatic, 1 = never, 2 = wherever the block layout allows it.  For
+    tests."""
+    _check(load_library().dg_force_tail_split(int(mode)), "dg_force_tail_split")

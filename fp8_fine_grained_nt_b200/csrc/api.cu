@@ -98,11 +98,14 @@ std::atomic<int> g_num_sms_limit{0};
 std::atomic<uint32_t> g_forced{0};
 
 // swap: 0 = automatic, 1 = never the small-M (swap-AB) kernel, 2 = always
-// where it applies (dense calls with M <= 128).
+// where it applies (dense calls with M <= 256).  tail: 0 = automatic, 1 =
+// never move a dense call's last partial wave to the small-M kernel, 2 =
+// wherever the layout allows it.
 std::atomic<int> g_forced_swap{0};
+std::atomic<int> g_forced_tail{0};
 
 struct Forced {
-    int bm, bn, split, pair, swap;
+    int bm, bn, split, pair, swap, tail;
 };
 
 uint32_t pack_forced(int bm, int bn, int split, int pair)
@@ -114,7 +117,8 @@ Forced forced_config()
 {
     const uint32_t w = g_forced.load(std::memory_order_relaxed);
     return Forced{(int)(w & 0x3FF), (int)((w >> 10) & 0x3FF), (int)((w >> 20) & 0xF),
-                  (int)((w >> 24) & 0x3), g_forced_swap.load(std::memory_order_relaxed)};
+                  (int)((w >> 24) & 0x3), g_forced_swap.load(std::memory_order_relaxed),
+                  g_forced_tail.load(std::memory_order_relaxed)};
 }
 
 int device_info(DeviceInfo **out)
@@ -248,7 +252,7 @@ double kb_cost_factor(int mw, int bn, int halves)
 // (pipeline ramp, and the BF16 store, which grows with the tile's size);
 // split-K adds the cluster reduction.
 double estimate_cycles(const Problem &pb, int mw, int bn, int split, int pair, int stages, int sms,
-                       int *tiles_out)
+                       int *tiles_out, double *wave_out = nullptr)
 {
     (void)stages;
     const int bm = pair ? 256 : 128 * mw;
@@ -280,6 +284,8 @@ double estimate_cycles(const Problem &pb, int mw, int bn, int split, int pair, i
         tile += 800.0 + (double)bm * bn * 4.0 * split / 256.0 / split;
     if (tiles_out)
         *tiles_out = (int)(tiles > 0x7fffffff ? 0x7fffffff : tiles);
+    if (wave_out)
+        *wave_out = tile;
     return waves * tile;
 }
 
@@ -407,6 +413,7 @@ int choose(const Problem &pb, int sms, int max_smem, const Candidate **out_cand,
     cfg->split = best_split;
     cfg->cta_pair = best->pair ? 2 : 1;
     cfg->swap_ab = 0;
+    cfg->tail_tiles = 0;
     if (best_split > 1)
         cfg->grid = (int)tiles * best_split; // one tile per cluster
     else if (best->pair)
@@ -452,9 +459,9 @@ int cluster_capacity_model(int split, int sms)
 // (decode shape, 34 to 102 CTAs) a CTA takes in ~30 B/clk whatever the
 // number of CTAs, so more CTAs stream faster until (b) binds; plus set-up
 // and, with a cluster, the exchange of the partial tiles.
-double skinny_cycles(int N, int K, int mn, int split, int cap)
+double skinny_cycles(int M, int N, int K, int mn, int split, int cap)
 {
-    const long tiles = ceil_div(N, SKINNY_TILE_N);
+    const long tiles = (long)ceil_div(N, SKINNY_TILE_N) * ceil_div(M, mn);
     const int nkb = K / 128;
     const long waves = (tiles + cap - 1) / cap;
     const long active = (tiles < cap ? tiles : cap) * (long)split;
@@ -472,6 +479,7 @@ struct SkinnyChoice {
     int cand_index;
     SkinnyParams plan; // sizes, split, stages and shared-memory offsets
     int smem_bytes;
+    double cycles;     // the estimate it was chosen by
 };
 
 // Shared-memory plan of a small-M kernel: as many operand stages as fit, up to
@@ -485,6 +493,8 @@ bool skinny_plan(const Problem &pb, int mn, int split, int max_smem, SkinnyParam
     p.K = pb.K;
     p.nkb = pb.K / 128;
     p.n_tiles = ceil_div(pb.N, SKINNY_TILE_N);
+    p.m_blocks = ceil_div(pb.M, mn);
+    p.tiles = p.n_tiles * p.m_blocks;
     p.split = split;
     const int units = ceil_div(p.nkb, SKINNY_KB_PER_STAGE);
     const int unit_max = ceil_div(units, split);
@@ -528,12 +538,15 @@ int skinny_capacity(DeviceInfo *dev, int idx, int split, int sms)
 int choose_skinny(const Problem &pb, int sms, int max_smem, DeviceInfo *dev, SkinnyChoice *out)
 {
     const Forced forced = forced_config();
+    // the smallest MN >= M; for larger M the widest, over blocks of MN rows
     int idx = -1;
     for (int i = 0; i < kNumSkinny; ++i)
         if (kSkinny[i].mn >= pb.M && (idx < 0 || kSkinny[i].mn < kSkinny[idx].mn))
             idx = i;
     if (idx < 0)
-        return DG_ERR_UNSUPPORTED_SHAPE;
+        for (int i = 0; i < kNumSkinny; ++i)
+            if (idx < 0 || kSkinny[i].mn > kSkinny[idx].mn)
+                idx = i;
     const int nkb = pb.K / 128;
     double best = 0;
     bool found = false;
@@ -544,10 +557,11 @@ int choose_skinny(const Problem &pb, int sms, int max_smem, DeviceInfo *dev, Ski
         if (!skinny_plan(pb, kSkinny[idx].mn, split, max_smem, &p))
             continue;
         const int cap = skinny_capacity(dev, idx, split, sms);
-        const double cost = skinny_cycles(pb.N, pb.K, kSkinny[idx].mn, split, cap);
+        const double cost = skinny_cycles(pb.M, pb.N, pb.K, kSkinny[idx].mn, split, cap);
         if (!found || cost < best * (1 - 1e-9)) {
             found = true;
             best = cost;
+            out->cycles = cost;
             out->cand = &kSkinny[idx];
             out->cand_index = idx;
             out->plan = p;
@@ -558,13 +572,17 @@ int choose_skinny(const Problem &pb, int sms, int max_smem, DeviceInfo *dev, Ski
     return found ? DG_OK : DG_ERR_UNSUPPORTED_SHAPE;
 }
 
-// Dense calls with M <= 128 take the small-M kernel, unless the test hooks
-// turn it off or pin a tile shape or CTA pairs of the other kernels.
+// Dense calls with M <= 256 take the small-M kernel (M > 128 in blocks of
+// 128 rows: a 256-row call is two tiles per 128 columns of D, no split of K
+// needed to fill the SMs), unless the test hooks turn it off or pin a tile
+// shape or CTA pairs of the other kernels.
+constexpr int kSkinnyMaxM = 256;
+
 bool use_skinny(const Problem &pb)
 {
-    if (pb.kind != DG_KIND_DENSE || pb.M > SKINNY_MAX_M)
+    if (pb.kind != DG_KIND_DENSE || pb.M > kSkinnyMaxM)
         return false;
-    if ((long)ceil_div(pb.N, SKINNY_TILE_N) > 65535)
+    if ((long)ceil_div(pb.N, SKINNY_TILE_N) * ceil_div(pb.M, SKINNY_MAX_M) > 65535)
         return false; // grid.y limit
     const Forced f = forced_config();
     if (f.swap != 0)
@@ -578,8 +596,8 @@ void skinny_config(const SkinnyChoice &c, dg_config *cfg)
     cfg->block_m = c.cand->mn;
     cfg->block_n = SKINNY_TILE_N;
     cfg->stages = c.plan.stages;
-    cfg->num_tiles = c.plan.n_tiles;
-    cfg->grid = c.plan.n_tiles * c.plan.split;
+    cfg->num_tiles = c.plan.tiles;
+    cfg->grid = c.plan.tiles * c.plan.split;
     cfg->smem_bytes = c.smem_bytes;
     const int mn = c.cand->mn;
     const int nbuf = 512 / mn < MAX_TMEM_BUFS ? 512 / mn : MAX_TMEM_BUFS;
@@ -622,14 +640,27 @@ int check_common(const void *A, const float *sa, const void *B, const float *sb,
     return DG_OK;
 }
 
-// Dense call with M <= 128 through the small-M kernel.
-int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const void *A, const float *sa,
-               const void *B, const float *sb, void *D, cudaStream_t stream)
+// Operands of a dense call as the small-M kernel reads them: a whole call, or
+// a block of one (rows [row0, M) and columns [col0, N) of D: A from row row0,
+// B from row col0, the scales offset to match, D with the call's row stride).
+struct DenseView {
+    const void *A;
+    const float *sa;
+    long ld_sa;
+    const void *B;
+    const float *sb;
+    void *D;
+    long ld_d;
+};
+
+// Dense call with M <= 256 (or a block of one) through the small-M kernel.
+int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const DenseView &v, cudaStream_t stream)
 {
     SkinnyChoice ch;
     int st = choose_skinny(pb, sms, dev->max_smem, dev, &ch);
     if (st != DG_OK)
         return st;
+    const void *A = v.A, *B = v.B;
     CUtensorMap tmap_a, tmap_b;
     // A: [M][K] bytes, box MN rows x 128 (rows past M are zero-filled)
     if ((st = make_tmap_2d(&tmap_a, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, pb.K, pb.M, pb.K, 128,
@@ -653,16 +684,17 @@ int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const void *A, const
             return DG_ERR_CUDA;
     }
     SkinnyParams p = ch.plan;
-    p.sa = sa;
-    p.ld_sa = get_tma_aligned_size(pb.M, 4);
-    p.sb = sb;
-    p.D = static_cast<uint16_t *>(D);
+    p.sa = v.sa;
+    p.ld_sa = (int)v.ld_sa;
+    p.sb = v.sb;
+    p.D = static_cast<uint16_t *>(v.D);
+    p.ld_d = v.ld_d;
     p.status = dev->status;
     p.timeout_ns = wait_timeout_ns();
     // persistent clusters: no more than the SM bound (and the device) holds
     const int cap = skinny_capacity(dev, ch.cand_index, p.split, sms);
     const int by_sms = sms / p.split > 0 ? sms / p.split : 1;
-    int clusters = p.n_tiles;
+    int clusters = p.tiles;
     if (clusters > cap)
         clusters = cap;
     if (clusters > by_sms)
@@ -678,6 +710,65 @@ int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const void *A, const
     return ch.cand->launch(args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
+// The last wave of a dense call on the 128-row kernels, when only partly
+// filled (tiles not a multiple of the persistent grid), runs a whole tile
+// time on a few SMs while the rest idle.  Tiles are numbered with N fastest,
+// so when that wave's tiles all lie in the last M block and start on a
+// 128-column boundary (the granularity of sb), they form one block of D: the
+// last M block's rows (at most 256) by the remaining columns.  That block is
+// a small-M GEMM, which the small-M kernel spreads over the SMs with its K
+// range split over clusters; it runs after the main kernel, which then
+// computes whole waves only.  Taken when the small-M estimate (plus the gap
+// between two launches) is below the wave it replaces.
+struct TailSplit {
+    int main_tiles; // tiles left to the main kernel
+    int row0;       // the block's first row and column in D
+    int col0;
+    Problem sub;    // the block as a dense problem
+};
+
+constexpr double kLaunchGapCycles = 4000.0; // ~2 us between dependent launches
+
+bool plan_tail(const Problem &pb, const dg_config &cfg, int sms, int max_smem, DeviceInfo *dev,
+               TailSplit *out)
+{
+    const Forced f = forced_config();
+    if (pb.kind != DG_KIND_DENSE || cfg.split != 1 || cfg.cta_pair != 1 || cfg.swap_ab || f.tail == 1)
+        return false;
+    const long tiles = cfg.num_tiles, grid = cfg.grid;
+    if (grid <= 0)
+        return false;
+    const long full = tiles / grid * grid;
+    if (full == 0 || full == tiles)
+        return false;
+    const long m_blocks = ceil_div(pb.M, cfg.block_m), n_blocks = ceil_div(pb.N, cfg.block_n);
+    const long last_row_first = (m_blocks - 1) * n_blocks; // first tile of the last M block
+    if (full < last_row_first)
+        return false;
+    const long col0 = (full - last_row_first) * cfg.block_n;
+    const long row0 = (m_blocks - 1) * cfg.block_m;
+    if (col0 % 128 != 0 || col0 >= pb.N || pb.M - row0 > kSkinnyMaxM)
+        return false;
+    Problem sub{DG_KIND_DENSE, (int)(pb.M - row0), (int)(pb.N - col0), pb.K, 1, 0};
+    if ((long)ceil_div(sub.N, SKINNY_TILE_N) * ceil_div(sub.M, SKINNY_MAX_M) > 65535)
+        return false; // grid.y limit
+    SkinnyChoice ch;
+    if (choose_skinny(sub, sms, max_smem, dev, &ch) != DG_OK)
+        return false;
+    if (f.tail != 2) {
+        double wave = 0;
+        const int mw = cfg.block_m / 128;
+        estimate_cycles(pb, mw, cfg.block_n, 1, 0, cfg.stages, sms, nullptr, &wave);
+        if (ch.cycles + kLaunchGapCycles >= wave)
+            return false;
+    }
+    out->main_tiles = (int)full;
+    out->row0 = (int)row0;
+    out->col0 = (int)col0;
+    out->sub = sub;
+    return true;
+}
+
 // Shared launch path for the three forms.
 int run(const Problem &pb, const void *A, const float *sa, const void *B, const float *sb, void *D,
         const int *m_indices, const int *masked_m, cudaStream_t stream)
@@ -687,14 +778,18 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     if (st != DG_OK)
         return st;
     const int sms = effective_sms(dev);
-    if (use_skinny(pb))
-        return run_skinny(pb, dev, sms, A, sa, B, sb, D, stream);
+    if (use_skinny(pb)) {
+        const DenseView v{A, sa, get_tma_aligned_size(pb.M, 4), B, sb, D, pb.N};
+        return run_skinny(pb, dev, sms, v, stream);
+    }
     const Candidate *cand = nullptr;
     dg_config cfg;
     SmemPlan plan;
     st = choose(pb, sms, dev->max_smem, &cand, &cfg, &plan);
     if (st != DG_OK)
         return st;
+    TailSplit tail;
+    const bool has_tail = plan_tail(pb, cfg, sms, dev->max_smem, dev, &tail);
 
     const int nkb = pb.K / 128;
     const int nnb = ceil_div(pb.N, 128);
@@ -759,7 +854,7 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     p.nnb = nnb;
     p.m_blocks = ceil_div(pb.M, cfg.block_m);
     p.n_blocks = ceil_div(pb.N, cfg.block_n);
-    p.num_tiles = cfg.num_tiles;
+    p.num_tiles = has_tail ? tail.main_tiles : cfg.num_tiles;
     p.split = cfg.split;
     p.kb_chunk = ceil_div(nkb, cfg.split);
     p.stages = cfg.stages;
@@ -784,7 +879,15 @@ int run(const Problem &pb, const void *A, const float *sa, const void *B, const 
     args.cluster = cand->pair ? 2 : cfg.split;
     args.smem_bytes = cfg.smem_bytes;
     args.stream = stream;
-    return cand->launch(args) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+    if (cand->launch(args) != cudaSuccess)
+        return DG_ERR_CUDA;
+    if (!has_tail)
+        return DG_OK;
+    const size_t r0 = (size_t)tail.row0, c0 = (size_t)tail.col0;
+    const DenseView v{static_cast<const uint8_t *>(A) + r0 * (size_t)pb.K, sa + r0, ld_sa,
+                      static_cast<const uint8_t *>(B) + c0 * (size_t)pb.K, sb + (c0 / 128) * (size_t)nkb,
+                      static_cast<uint16_t *>(D) + r0 * (size_t)pb.N + c0, pb.N};
+    return run_skinny(tail.sub, dev, sms, v, stream);
 }
 
 } // namespace
@@ -988,7 +1091,7 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
         skinny_config(ch, out);
         const int cap = cluster_capacity_model(ch.plan.split, sms);
         const int by_sms = sms / ch.plan.split > 0 ? sms / ch.plan.split : 1;
-        int clusters = ch.plan.n_tiles < cap ? ch.plan.n_tiles : cap;
+        int clusters = ch.plan.tiles < cap ? ch.plan.tiles : cap;
         clusters = clusters < by_sms ? clusters : by_sms;
         out->grid = clusters * ch.plan.split;
         return DG_OK;
@@ -996,9 +1099,14 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
     const Candidate *cand = nullptr;
     SmemPlan plan;
     const int st = choose(pb, sms, kDefaultMaxSmem, &cand, out, &plan);
-    if (st == DG_OK)
-        out->swap_ab = 0;
-    return st;
+    if (st != DG_OK)
+        return st;
+    out->swap_ab = 0;
+    out->tail_tiles = 0;
+    TailSplit tail;
+    if (plan_tail(pb, *out, sms, kDefaultMaxSmem, nullptr, &tail))
+        out->tail_tiles = out->num_tiles - tail.main_tiles;
+    return DG_OK;
 }
 
 int dg_force_config(int block_m, int block_n, int split, int cta_pair)
@@ -1027,6 +1135,14 @@ int dg_force_swap_ab(int mode)
     if (mode < 0 || mode > 2)
         return DG_ERR_INVALID_ARGUMENT;
     g_forced_swap.store(mode, std::memory_order_relaxed);
+    return DG_OK;
+}
+
+int dg_force_tail_split(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return DG_ERR_INVALID_ARGUMENT;
+    g_forced_tail.store(mode, std::memory_order_relaxed);
     return DG_OK;
 }
 

@@ -75,6 +75,13 @@ struct KernelTraits {
     // buffers released together, which amortises the per-block handshake.
     static constexpr int GROUP_BY_REGS = PREFETCH ? 64 / COLS_PER_THREAD : 1;
     static constexpr int GROUP = GROUP_BY_REGS < NBUF / 2 ? GROUP_BY_REGS : (NBUF / 2 > 0 ? NBUF / 2 : 1);
+    // Wide tiles (two epilogue warpgroups, each owning BN / 2 columns of
+    // every row, read in two batches): each K block is issued as two MMAs of
+    // N = BN / 2, one per warpgroup's columns, each half with its own
+    // completion and release barriers, so that the MMAs into one half of a
+    // buffer wait only for the warpgroup that reads that half.
+    static constexpr bool HALVES = MW == 1 && !PAIR && !SCALAR && !PREFETCH;
+    static_assert(!HALVES || (BN / 2) % 16 == 0, "an M = 128 MMA takes N in multiples of 16");
     static constexpr uint32_t A_HALF_BYTES = HALF_M * BLOCK_K;
     static constexpr uint32_t B_BYTES = B_ROWS * BLOCK_K;
     static_assert(NBUF >= 2 && NBUF <= MAX_TMEM_BUFS && TMEM_NEED <= 512, "TMEM holds 512 columns");
@@ -124,8 +131,21 @@ struct TileInfo {
     int d_row0;  // row of D (all groups flattened) holding row m0
 };
 
+// Contiguous form: the expert of tile t's M block (m_indices of its first
+// row), or 0 for the other forms and for t past the last tile.
 template <int MW, int BN, bool PAIR>
-__device__ __forceinline__ TileInfo get_tile(const Params &p, int t, const int *prefix, int pair_rank)
+__device__ __forceinline__ int expert_of_tile(const Params &p, int t, int num_tiles)
+{
+    if (p.kind != KIND_CONTIGUOUS || t >= num_tiles)
+        return 0;
+    constexpr int BM = KernelTraits<MW, BN, PAIR>::BLOCK_M;
+    return __ldg(p.m_indices + (t / p.n_blocks) * BM);
+}
+
+// Tile t of this CTA's walk; `e` is the tile's expert for the contiguous form
+// (expert_of_tile, read ahead by the caller).
+template <int MW, int BN, bool PAIR>
+__device__ __forceinline__ TileInfo get_tile(const Params &p, int t, const int *prefix, int pair_rank, int e)
 {
     constexpr int BM = KernelTraits<MW, BN, PAIR>::BLOCK_M;
     TileInfo ti;
@@ -165,7 +185,6 @@ __device__ __forceinline__ TileInfo get_tile(const Params &p, int t, const int *
         ti.g = 0;
         ti.b_row0 = nb * BN;
         if (p.kind == KIND_CONTIGUOUS) {
-            const int e = __ldg(p.m_indices + ti.m0);
             if (e < 0 || e >= p.num_groups) {
                 if (e >= p.num_groups)
                     atomicOr(p.status, DEVERR_BAD_INDEX);
@@ -348,6 +367,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t *sa_empty = sa_full + 2;
     uint64_t *mma_done = sa_empty + 2;
     uint64_t *tile_full = mma_done + 1; // per-tensor scaling: a tile's accumulator is complete (x2)
+    // split MMAs (T::HALVES): done_lo[j]: the first column half of K block
+    // j is complete (done[j] then covers the second half and frees the
+    // stage); tmem_empty[b] / tmem_empty_hi[b]: the first / second
+    // warpgroup has read its half of buffer b
+    uint64_t *done_lo = tile_full + 2;
+    uint64_t *tmem_empty_hi = done_lo + DONE_RING;
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + plan.off_misc);
     volatile uint32_t *abort_flag = misc + 1;
     int *prefix = reinterpret_cast<int *>(smem + plan.off_prefix);
@@ -362,9 +387,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int j = 0; j < DONE_RING; ++j)
             mbar_init(&done[j], 1);
         for (int b = 0; b < T::NBUF; ++b) {
-            // a pair's leader also counts the peer's epilogue warps
-            mbar_init(&tmem_empty[b], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
+            // a pair's leader also counts the peer's epilogue warps; split
+            // MMAs: one warpgroup per half
+            mbar_init(&tmem_empty[b], PAIR ? 2 * NUM_EPI_WARPS : (T::HALVES ? 4 : NUM_EPI_WARPS));
+            if constexpr (T::HALVES)
+                mbar_init(&tmem_empty_hi[b], 4);
         }
+        if constexpr (T::HALVES)
+            for (int j = 0; j < DONE_RING; ++j)
+                mbar_init(&done_lo[j], 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sb_full[b], 32);
             mbar_init(&sb_empty[b], NUM_EPI_WARPS);
@@ -453,8 +484,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool a_side = warp == 0;
         uint32_t it = 0, s = 0;
         bool ok = true;
+        // the next tile's expert (contiguous form: a global read) is read
+        // one tile ahead, so that it overlaps this tile
+        int e_next = expert_of_tile<MW, BN, PAIR>(p, t_first, num_tiles);
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank, e_next);
+            e_next = expert_of_tile<MW, BN, PAIR>(p, t + t_stride, num_tiles);
             if (!ti.valid)
                 continue;
             // A: lanes 0..halves-1 copy the 128-row halves; B: lane 0
@@ -520,8 +555,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // TMEM buffer (tile mod 2); one commit per K block frees its
                 // stage, one more at the last K block publishes the tile.
                 uint32_t tile_it = 0;
+                // the next tile's expert (contiguous form: a global read) is read
+                // one tile ahead, so that it overlaps this tile
+                int e_next = expert_of_tile<MW, BN, PAIR>(p, t_first, num_tiles);
                 for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-                    const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+                    const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank, e_next);
+                    e_next = expert_of_tile<MW, BN, PAIR>(p, t + t_stride, num_tiles);
                     if (!ti.valid)
                         continue;
                     const uint32_t buf = tile_it & 1;
@@ -553,8 +592,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ++tile_it;
                 }
             }
+            // the next tile's expert (contiguous form: a global read) is read
+            // one tile ahead, so that it overlaps this tile
+            int e_next = expert_of_tile<MW, BN, PAIR>(p, t_first, num_tiles);
             for (int t = t_first; !SCALAR && ok && t < num_tiles; t += t_stride) {
-                const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+                const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank, e_next);
+                e_next = expert_of_tile<MW, BN, PAIR>(p, t + t_stride, num_tiles);
                 if (!ti.valid)
                     continue;
                 const int halves = (MW == 1) ? 1 : (ti.rows > HALF_M ? 2 : 1);
@@ -582,16 +625,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     const uint64_t a_desc = a_desc0 + s * stage_step;
                     const uint64_t b_desc = b_desc0 + s * stage_step;
-                    for (int h = 0; h < halves; ++h) {
-                        const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS + h * BN);
+                    if constexpr (T::HALVES) {
+                        // columns [0, BN/2) (B rows [0, BN/2)), then [BN/2, BN)
+                        // once the second warpgroup has read its half
+                        constexpr uint32_t idesc_h = make_idesc(BN / 2);
+                        const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS);
 #pragma unroll
-                        for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
-                            const uint64_t ad = a_desc + (uint64_t)((h * T::A_HALF_BYTES + k * MMA_K) >> 4);
-                            const uint64_t bd = b_desc + (uint64_t)((k * MMA_K) >> 4);
-                            if constexpr (PAIR)
-                                mma_f8f6f4_pair(d, ad, bd, idesc, k > 0 ? 1u : 0u);
-                            else
-                                mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
+                            mma_f8f6f4(d, a_desc + (uint64_t)((k * MMA_K) >> 4),
+                                       b_desc + (uint64_t)((k * MMA_K) >> 4), idesc_h, k > 0 ? 1u : 0u);
+                        mma_commit(&done_lo[kb_it % DONE_RING]);
+                        if (!wait_bar(&tmem_empty_hi[buf], ((kb_it / T::NBUF) & 1) ^ 1, abort_flag, p)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // B rows from BN/2 on: BN/2 is a multiple of 8, so the
+                        // half starts on a 1024-byte swizzle atom
+                        const uint64_t b_hi = b_desc + (uint64_t)((BN / 2 * BLOCK_K) >> 4);
+#pragma unroll
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
+                            mma_f8f6f4(d + (uint32_t)(BN / 2), a_desc + (uint64_t)((k * MMA_K) >> 4),
+                                       b_hi + (uint64_t)((k * MMA_K) >> 4), idesc_h, k > 0 ? 1u : 0u);
+                    } else {
+                        for (int h = 0; h < halves; ++h) {
+                            const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS + h * BN);
+#pragma unroll
+                            for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
+                                const uint64_t ad = a_desc + (uint64_t)((h * T::A_HALF_BYTES + k * MMA_K) >> 4);
+                                const uint64_t bd = b_desc + (uint64_t)((k * MMA_K) >> 4);
+                                if constexpr (PAIR)
+                                    mma_f8f6f4_pair(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                                else
+                                    mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                            }
                         }
                     }
                     // one commit per K block frees its stage and publishes its
@@ -625,8 +692,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         regs_dec<REGS_PRODUCER>();
         uint32_t tile_it = 0, grp_it = 0;
         bool ok = true;
+        // the next tile's expert (contiguous form: a global read) is read
+        // one tile ahead, so that it overlaps this tile
+        int e_next = expert_of_tile<MW, BN, PAIR>(p, t_first, num_tiles);
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank, e_next);
+            e_next = expert_of_tile<MW, BN, PAIR>(p, t + t_stride, num_tiles);
             if (!ti.valid)
                 continue;
             const int slot = tile_it & 1;
@@ -679,12 +750,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         uint32_t kb_it = 0, tile_it = 0, sa_it = 0;
         bool ok = true;
+        // the next tile's expert (contiguous form: a global read) is read
+        // one tile ahead, so that it overlaps this tile
+        int e_next = expert_of_tile<MW, BN, PAIR>(p, t_first, num_tiles);
         for (int t = t_first; ok && t < num_tiles; t += t_stride) {
-            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank);
+            const TileInfo ti = get_tile<MW, BN, PAIR>(p, t, prefix, pair_rank, e_next);
+            e_next = expert_of_tile<MW, BN, PAIR>(p, t + t_stride, num_tiles);
             if (!ti.valid)
                 continue;
             const bool active = (MW == 1) ? true : (half * HALF_M < ti.rows);
             const int cbase = ti.n0 + col0;
+            // contiguous form: the expert of this thread's row, read now (a
+            // global read) and checked when the tile is stored
+            int row_expert = 0;
+            if (p.kind == KIND_CONTIGUOUS && active && row_in_tile < ti.rows)
+                row_expert = __ldg(p.m_indices + ti.d_row0 + row_in_tile);
             float acc[NC];
             if constexpr (SCALAR) {
                 // Per-tensor scaling: read the tile's accumulator once, scale
@@ -751,9 +831,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             auto buf_addr = [&](uint32_t it) {
                 return t_lane + (uint32_t)((int)(it % T::NBUF) * T::BUF_COLS);
             };
+            // split MMAs: the first warpgroup's half completes (and is
+            // released) on barriers of its own
+            uint64_t *const my_done = (T::HALVES && wg == 0) ? done_lo : done;
+            uint64_t *const my_empty = (T::HALVES && wg == 1) ? tmem_empty_hi : tmem_empty;
             // wait for K block `it`'s partial in TMEM
             auto wait_full = [&](uint32_t it) {
-                const bool r = wait_bar_warp(&done[it % DONE_RING], (it / DONE_RING) & 1, abort_flag, p);
+                const bool r = wait_bar_warp(&my_done[it % DONE_RING], (it / DONE_RING) & 1, abort_flag, p);
                 tc_fence_after();
                 return r;
             };
@@ -763,7 +847,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0)
                     for (int j = 0; j < cnt; ++j) {
-                        uint64_t *bar = &tmem_empty[(it + j) % T::NBUF];
+                        uint64_t *bar = &my_empty[(it + j) % T::NBUF];
                         if (PAIR && !leader)
                             mbar_arrive_cluster(map_shared_rank(smem_addr(bar), 0u));
                         else
@@ -891,7 +975,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // ---- store the tile's rows as BF16
             bool row_ok = active && row_in_tile < ti.rows;
             if (row_ok && p.kind == KIND_CONTIGUOUS) {
-                const int e = __ldg(p.m_indices + ti.d_row0 + row_in_tile);
+                const int e = row_expert;
                 if (e != ti.g) {
                     row_ok = false;
                     if (e >= 0)
@@ -1009,7 +1093,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // sums rows [r, r + BLOCK_M / split) of all partials in rank order
         // (deterministic) through distributed shared memory and stores them.
         cluster_sync();
-        const TileInfo ti = get_tile<MW, BN, PAIR>(p, t_first, prefix, pair_rank);
+        const TileInfo ti = get_tile<MW, BN, PAIR>(p, t_first, prefix, pair_rank,
+                                                   expert_of_tile<MW, BN, PAIR>(p, t_first, num_tiles));
         const int rows_per = T::BLOCK_M / p.split;
         const int r0 = split_rank * rows_per;
         constexpr int CHUNKS = BN / 8;

@@ -143,23 +143,24 @@ __device__ __forceinline__ void skinny_promote(float (&acc)[NC], const float *v,
 }
 
 // The scales of one tile for a CTA's K blocks, as asynchronous copies by one
-// warp: sa[kb][m] for m < M (zero-filled up to MN) and sb[tile][kb].
+// warp: sa[kb][m0 + m] for m < rows (zero-filled up to MN) and sb[nt][kb].
 template <int MN>
 __device__ __forceinline__ void skinny_copy_scales(const SkinnyParams &p, float *sa_s, float *sb_s,
-                                                   int tile, int kb_lo, int cnt, int lane)
+                                                   int nt, int m0, int rows, int kb_lo, int cnt, int lane)
 {
     constexpr int C4 = MN / 4; // 16-byte chunks per K block
     for (int idx = lane; idx < cnt * C4; idx += 32) {
         const int i = idx / C4;
         const int m = (idx - i * C4) * 4;
-        const int avail = p.M - m;
+        const int avail = rows - m;
         const uint32_t bytes = avail >= 4 ? 16u : (avail > 0 ? 4u * (uint32_t)avail : 0u);
-        // a chunk past M reads nothing (a valid address is still given)
-        const float *src = p.sa + (size_t)(kb_lo + i) * p.ld_sa + (bytes ? m : 0);
+        // a chunk past the tile's rows reads nothing (a valid address is still
+        // given; m0 is a multiple of MN, so every source chunk is 16-byte aligned)
+        const float *src = p.sa + (size_t)(kb_lo + i) * p.ld_sa + m0 + (bytes ? m : 0);
         cp_async_16_zfill(sa_s + i * MN + m, src, bytes);
     }
     for (int i = lane; i < cnt; i += 32)
-        cp_async_4(sb_s + i, p.sb + (size_t)tile * p.nkb + kb_lo + i);
+        cp_async_4(sb_s + i, p.sb + (size_t)nt * p.nkb + kb_lo + i);
 }
 
 template <int MN>
@@ -199,32 +200,42 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     constexpr int G = SKINNY_KB_PER_STAGE;
     const int rank = p.split > 1 ? (int)cluster_ctarank() : 0;
     const int units = (p.nkb + G - 1) / G;
-    const int kb_lo = G * (int)((long)rank * units / p.split);
-    const int kb_hi = min(p.nkb, G * (int)((long)(rank + 1) * units / p.split));
+    // (32-bit products: units < 2^24 and rank < 8)
+    const int kb_lo = G * (int)((uint32_t)rank * (uint32_t)units / (uint32_t)p.split);
+    const int kb_hi = min(p.nkb, G * (int)((uint32_t)(rank + 1) * (uint32_t)units / (uint32_t)p.split));
     const int cnt = max(0, kb_hi - kb_lo);
     const int ucnt = (cnt + G - 1) / G; // stages per tile
     const int t_first = (int)blockIdx.y;
     const int t_stride = (int)gridDim.y;
+    // tile t: B rows [128 * (t / m_blocks), +128), A rows [MN * (t % m_blocks),
+    // +MN) (the A blocks of one B block are neighbours: B is read from HBM
+    // once and from L2 after); rows = A rows of the tile that exist
+    auto tile_rows = [&](int t) { return min(MN, p.M - MN * (t % p.m_blocks)); };
     // the output items (one row m, 8 consecutive columns) of a tile that CTA
     // r of the cluster sums and stores: [r * items / split, (r + 1) * items / split)
-    const int items = p.M * (SKINNY_TILE_N / 8);
-    auto item_lo = [&](int r) { return (int)((long)r * items / p.split); };
-    const uint32_t slot_bytes = skinny_recv_slot_items(p.M, p.split) * 32u;
-    const uint32_t my_bytes = (uint32_t)(item_lo(rank + 1) - item_lo(rank)) * 32u;
+    auto item_lo = [&](int items, int r) {
+        return (int)((uint32_t)r * (uint32_t)items / (uint32_t)p.split); // items <= 2048, r <= 8
+    };
+    const uint32_t slot_bytes = skinny_recv_slot_items(min(MN, p.M), p.split) * 32u;
+    auto my_bytes = [&](int t) {
+        const int items = tile_rows(t) * (SKINNY_TILE_N / 8);
+        return (uint32_t)(item_lo(items, rank + 1) - item_lo(items, rank)) * 32u;
+    };
 
     // warp 0 copies B, warp 3 copies A into stage s (each with its bytes):
     // K blocks [kb, kb + G) (any past K are zero-filled and not used)
     const bool b_side = warp == 0;
-    auto issue_load = [&](int s, int kb, int n0) {
+    auto issue_load = [&](int s, int kb, int t) {
         uint8_t *dst = smem + (uint32_t)s * p.stage_bytes;
         if (b_side) {
             mbar_arrive_expect_tx(&full[s], G * T::B_BYTES);
-            tma_load_4d(dst, &tmap_b, &full[s], 0, 0, kb, n0 / 8);
+            tma_load_4d(dst, &tmap_b, &full[s], 0, 0, kb, (t / p.m_blocks) * (SKINNY_TILE_N / 8));
         } else {
             mbar_arrive_expect_tx(&full[s], G * T::A_BYTES);
 #pragma unroll
             for (int z = 0; z < G; ++z)
-                tma_load_2d(dst + G * T::B_BYTES + z * T::A_BYTES, &tmap_a, &full[s], (kb + z) * BLOCK_K, 0);
+                tma_load_2d(dst + G * T::B_BYTES + z * T::A_BYTES, &tmap_a, &full[s], (kb + z) * BLOCK_K,
+                            MN * (t % p.m_blocks));
         }
     };
     // the last K block (counted over this CTA's tiles) that stage use u holds
@@ -241,7 +252,7 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     // programmatic dependent launch, this set-up overlaps the end of the
     // previous kernel: no thread touches global memory (the operands may be
     // that kernel's output, D its input) before the dependency wait.
-    const int first = (t_first < p.n_tiles) ? (ucnt < stages ? ucnt : stages) : 0;
+    const int first = (t_first < p.tiles) ? (ucnt < stages ? ucnt : stages) : 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s)
             mbar_init(&full[s], 2);
@@ -258,7 +269,7 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
         named_barrier_sync(1, 64); // the stage barriers are initialised
         if (lane == 0)
             for (int i = 0; i < first; ++i)
-                issue_load(i, kb_lo + G * i, t_first * SKINNY_TILE_N);
+                issue_load(i, kb_lo + G * i, t_first);
     }
     if (threadIdx.x == 0) {
         for (int j = 0; j < DONE_RING; ++j)
@@ -269,32 +280,40 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
         mbar_init(mma_done, 1);
         mbar_init(recv_full, 1);
         // the first tile's slices from the cluster: expected before any can arrive
-        if (p.split > 1 && t_first < p.n_tiles)
-            mbar_arrive_expect_tx(recv_full, (uint32_t)p.split * my_bytes);
+        if (p.split > 1 && t_first < p.tiles)
+            mbar_arrive_expect_tx(recv_full, (uint32_t)p.split * my_bytes(t_first));
         misc[1] = 0u;
         fence_mbarrier_init();
     }
-    if (warp == 2 && t_first < p.n_tiles)
-        skinny_copy_scales<MN>(p, sa_s, sb_s, t_first, kb_lo, cnt, lane);
+    if (warp == 2 && t_first < p.tiles)
+        skinny_copy_scales<MN>(p, sa_s, sb_s, t_first / p.m_blocks, MN * (t_first % p.m_blocks),
+                               tile_rows(t_first), kb_lo, cnt, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     // the next kernel may start its own set-up on SMs this grid leaves free
     grid_launch_dependents();
-    // the cluster's barriers are initialised before any CTA sends a slice:
-    // arrive now, wait before the first send (the initialisation is ordered
-    // by fence.mbarrier_init; a releasing arrive would also wait for this
-    // thread's earlier memory operations)
-    if (p.split > 1)
+    // the cluster's barriers are initialised before any CTA sends a slice
+    // (the initialisation is ordered by fence.mbarrier_init; a releasing
+    // arrive would also wait for this thread's earlier memory operations).
+    // The cluster's CTAs start together, and every role's first wait (for
+    // data, MMAs or scales) is longer than this barrier.
+    if (p.split > 1) {
         cluster_arrive_relaxed();
+        cluster_wait();
+    }
 
+    bool mma_done_committed = false; // (MMA issuer)
+    bool cluster_wait_pending = false; // arrived on the closing cluster barrier
     uint32_t g0 = 0; // this CTA's K blocks of earlier tiles (ring position)
     uint32_t u0 = 0; // this CTA's stage uses of earlier tiles
     int tile_it = 0;
-    for (int tile = t_first; tile < p.n_tiles;
+    for (int tile = t_first; tile < p.tiles;
          tile += t_stride, g0 += (uint32_t)cnt, u0 += (uint32_t)ucnt, ++tile_it) {
-        const int n0 = tile * SKINNY_TILE_N;
+        const int n0 = (tile / p.m_blocks) * SKINNY_TILE_N;
+        const int m0 = MN * (tile % p.m_blocks);
+        const int rows = tile_rows(tile);
         if (warp == 0 || warp == 3) {
             // -------------------------------------------------------- producers
             if (lane == 0) {
@@ -308,7 +327,7 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                         if (!skinny_wait(&done[j % DONE_RING], (j / DONE_RING) & 1u, abort_flag, p))
                             break;
                     }
-                    issue_load(s, kb_lo + G * (int)(u - u0), n0);
+                    issue_load(s, kb_lo + G * (int)(u - u0), tile);
                     issued = u + 1;
                 }
                 // every copy issued must land before the ring is reused for
@@ -355,13 +374,19 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                         mma_commit(&done[g % DONE_RING]);
                     }
                 }
+                // after the CTA's last MMAs: the "all MMAs done" barrier,
+                // awaited before TMEM is released at the end
+                if (tile + t_stride >= p.tiles) {
+                    mma_commit(mma_done);
+                    mma_done_committed = true;
+                }
             }
         } else if (warp == 2) {
             // -------------------------------------------------------- scales
             // the tile's scale copies (the first tile's were started at entry;
             // the previous tile's have been read: the end-of-tile barriers)
             if (tile_it > 0)
-                skinny_copy_scales<MN>(p, sa_s, sb_s, tile, kb_lo, cnt, lane);
+                skinny_copy_scales<MN>(p, sa_s, sb_s, tile / p.m_blocks, m0, rows, kb_lo, cnt, lane);
             cp_async_mbar_arrive_noinc(scales_full);
         } else if (warp >= 4) {
             // -------------------------------------------------------- epilogue
@@ -425,23 +450,20 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                         }
                     }
                 } else {
-                    // the partial in two halves, each loaded, waited for and
-                    // promoted in turn (registers are fewer at 384 threads)
-                    constexpr int CH = NC / 2;
-                    float v[CH];
+                    // the whole partial loaded at once (one wait), its buffer
+                    // handed back, then promoted (registers are fewer at 384
+                    // threads: no next partial in flight)
+                    float v[NC];
                     for (int i = 0; ok && i < cnt; ++i) {
                         const uint32_t g = g0 + (uint32_t)i;
                         if (!wait_done(g)) {
                             ok = false;
                             break;
                         }
-                        tmem_issue_p<CH>(buf_addr(g), v);
-                        tmem_wait_tie<CH>(v);
-                        skinny_promote<NC, 0, CH>(acc, v, sa_s + i * MN + col0, sb_s[i]);
-                        tmem_issue_p<CH>(buf_addr(g) + (uint32_t)CH, v);
-                        tmem_wait_tie<CH>(v);
+                        tmem_issue_p<NC>(buf_addr(g), v);
+                        tmem_wait_tie<NC>(v);
                         release(g);
-                        skinny_promote<NC, CH, CH>(acc, v, sa_s + i * MN + col0, sb_s[i]);
+                        skinny_promote<NC, 0, NC>(acc, v, sa_s + i * MN + col0, sb_s[i]);
                     }
                 }
             }
@@ -462,19 +484,18 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
         // ------------------------------------------------------------ reduce + store
         __syncthreads(); // the partial tile is complete
         const uint32_t red_local = smem_addr(smem);
-        const int lo = item_lo(rank), hi = item_lo(rank + 1);
+        const int items = rows * (SKINNY_TILE_N / 8);
+        const int lo = item_lo(items, rank), hi = item_lo(items, rank + 1);
         if (p.split > 1) {
             // Send slice r of this CTA's partial tile (items of CTA r) to CTA
             // r's receive area, slot `rank`; wait for the tile's slices from
             // every CTA, sum them in rank order, store.  The receive area is
             // this CTA's own shared memory outside the operand ring, free
             // since the previous tile's closing cluster barrier.
-            if (tile_it == 0)
-                cluster_wait();
             if (threadIdx.x < p.split) {
                 // lane r of warp 0 sends slice r (the copies are issued in parallel)
                 const int r = (int)threadIdx.x;
-                const int rlo = item_lo(r), rhi = item_lo(r + 1);
+                const int rlo = item_lo(items, r), rhi = item_lo(items, r + 1);
                 const uint32_t recv_local = smem_addr(smem + p.off_recv) + (uint32_t)rank * slot_bytes;
                 if (rhi > rlo)
                     bulk_copy_to_cluster(map_shared_rank(recv_local, (uint32_t)r),
@@ -482,6 +503,17 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                                          map_shared_rank(smem_addr(recv_full), (uint32_t)r));
             }
             const bool got = hi <= lo || skinny_wait(recv_full, (uint32_t)tile_it & 1u, abort_flag, p);
+            const bool last = tile + t_stride >= p.tiles;
+            if (last) {
+                // Every slice sent to this CTA has landed.  Once every CTA
+                // has said so, every copy that read this CTA's partial tile
+                // has completed and the CTA may exit: the wait is left for
+                // the very end, after the sums, the stores and the TMEM
+                // release.
+                __syncwarp();
+                cluster_arrive();
+                cluster_wait_pending = true;
+            }
             const float *recv = reinterpret_cast<const float *>(smem + p.off_recv);
             for (int it = lo + (int)threadIdx.x; got && it < hi; it += T::THREADS) {
                 const int m = it >> 4;
@@ -497,18 +529,22 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                     sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
                     sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
                 }
-                st_global_v4(p.D + (size_t)m * p.N + n, pack_bf16x2(sum[0], sum[1]),
+                st_global_v4(p.D + (size_t)(m0 + m) * (size_t)p.ld_d + n, pack_bf16x2(sum[0], sum[1]),
                              pack_bf16x2(sum[2], sum[3]), pack_bf16x2(sum[4], sum[5]),
                              pack_bf16x2(sum[6], sum[7]));
             }
-            __syncthreads(); // every thread has read the receive area
-            // the next tile's slices are expected before any can be sent
-            if (threadIdx.x == 0 && tile + t_stride < p.n_tiles && hi > lo)
-                mbar_arrive_expect_tx(recv_full, (uint32_t)p.split * my_bytes);
-            // every CTA has received all its slices (so every copy that read
-            // this CTA's partial tile has completed): the rings can be reused
-            // and no CTA leaves while a copy into it is in flight
-            cluster_sync();
+            if (!last) {
+                __syncthreads(); // every thread has read the receive area
+                // the next tile's slices are expected before any can be sent
+                if (threadIdx.x == 0) {
+                    const uint32_t next_bytes = my_bytes(tile + t_stride);
+                    if (next_bytes > 0)
+                        mbar_arrive_expect_tx(recv_full, (uint32_t)p.split * next_bytes);
+                }
+                // every CTA has received all its slices and read them: the
+                // rings and the receive areas can be reused
+                cluster_sync();
+            }
         } else {
             for (int it = lo + (int)threadIdx.x; it < hi; it += T::THREADS) {
                 const int m = it >> 4;
@@ -519,18 +555,17 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                 const uint32_t off = (uint32_t)(m * SKINNY_TILE_N + c8) * 4u;
                 const float4 a = *reinterpret_cast<const float4 *>(smem + off);
                 const float4 b = *reinterpret_cast<const float4 *>(smem + off + 16);
-                st_global_v4(p.D + (size_t)m * p.N + n, pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                st_global_v4(p.D + (size_t)(m0 + m) * (size_t)p.ld_d + n, pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
                              pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
             }
             __syncthreads(); // the ring is reused by the next tile
         }
     }
-    if (p.split > 1 && t_first >= p.n_tiles)
-        cluster_wait(); // pairs the set-up arrival
     if (warp == 1) {
         if (lane == 0) {
             // all MMAs complete before TMEM is released
-            mma_commit(mma_done);
+            if (!mma_done_committed)
+                mma_commit(mma_done);
             skinny_drain(mma_done, 0, abort_flag, p);
         }
         __syncwarp();
@@ -539,6 +574,8 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
     }
     if (warp == 2)
         cp_async_wait_all(); // no scale copy outlives the CTA
+    if (cluster_wait_pending)
+        cluster_wait(); // no copy reads this CTA's shared memory any more
 }
 
 } // namespace fp8nt

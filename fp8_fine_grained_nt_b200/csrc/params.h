@@ -111,8 +111,9 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     p.off_bars = align_up_u32(off, 8);
     // full per stage, the ring of "K block done" barriers, TMEM empty per
     // partial buffer, sb and sa full/empty x2, one "all MMAs done" barrier,
-    // two "tile accumulated" barriers (per-tensor scaling)
-    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u + 2u);
+    // two "tile accumulated" barriers (per-tensor scaling), and for MMAs
+    // split in column halves a second done ring and TMEM-empty set
+    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u + 2u + DONE_RING + MAX_TMEM_BUFS);
     p.off_misc = align_up_u32(off, 16);
     p.total = p.off_misc + 16;
     return p;
@@ -132,11 +133,13 @@ constexpr int SKINNY_MAX_M = 128;
 constexpr int SKINNY_KB_PER_STAGE = 2;
 
 struct SkinnyParams {
-    int M;          // rows of A and D (<= MN of the kernel)
+    int M;          // rows of A and D
     int N;
     int K;
     int nkb;        // K / 128
-    int n_tiles;    // ceil(N / 128)
+    int n_tiles;    // ceil(N / 128): 128-row blocks of B
+    int m_blocks;   // ceil(M / MN): blocks of MN rows of A
+    int tiles;      // n_tiles * m_blocks (tile t: B block t / m_blocks, A block t % m_blocks)
     int split;      // CTAs of a cluster that share one tile, each a contiguous K range
                     // (whole stages of SKINNY_KB_PER_STAGE K blocks)
     int kb_max;     // K blocks of the largest share
@@ -153,7 +156,8 @@ struct SkinnyParams {
     const float *sa;      // [K/128][ld_sa]
     int ld_sa;
     const float *sb;      // [ceil(N/128)][K/128]
-    uint16_t *D;          // [M][N] BF16 bits
+    uint16_t *D;          // [M][ld_d] BF16 bits (the first N columns are written)
+    long ld_d;            // row stride of D in elements (>= N, a multiple of 8)
     unsigned int *status;
     uint64_t timeout_ns;
 };
@@ -167,9 +171,9 @@ constexpr int SKINNY_NUM_BARS_FIXED = DONE_RING + MAX_TMEM_BUFS + 3;
 // slices of the output that the cluster's CTAs send to one CTA: split slots
 // of ceil(items / split) items, an item being 8 FP32 values (items = 16 M).
 __host__ __device__ inline uint32_t skinny_red_bytes(int mn) { return (uint32_t)mn * SKINNY_TILE_N * 4u; }
-__host__ __device__ inline uint32_t skinny_recv_slot_items(int m, int split)
+__host__ __device__ inline uint32_t skinny_recv_slot_items(int rows, int split)
 {
-    const uint32_t items = (uint32_t)m * (SKINNY_TILE_N / 8);
+    const uint32_t items = (uint32_t)rows * (SKINNY_TILE_N / 8);
     return (items + (uint32_t)split - 1) / (uint32_t)split;
 }
 
@@ -181,7 +185,8 @@ __host__ __device__ inline void make_skinny_plan(SkinnyParams &p, int mn, int st
     const uint32_t red = skinny_red_bytes(mn);
     p.region = ring > red ? ring : red;
     p.off_recv = align_up_u32(p.region, 1024);
-    const uint32_t recv = p.split > 1 ? (uint32_t)p.split * skinny_recv_slot_items(p.M, p.split) * 32u : 0u;
+    const int rows = p.M < mn ? p.M : mn; // rows of the largest tile
+    const uint32_t recv = p.split > 1 ? (uint32_t)p.split * skinny_recv_slot_items(rows, p.split) * 32u : 0u;
     p.off_sa = align_up_u32(p.off_recv + recv, 128);
     p.off_sb = p.off_sa + (uint32_t)p.kb_max * (uint32_t)mn * 4u;
     p.off_bars = align_up_u32(p.off_sb + (uint32_t)p.kb_max * 4u, 8);

@@ -15,9 +15,10 @@
 //
 // HBM-bound: one warp per 32 rows x 128 columns, 8 lanes per row, each lane
 // 16 consecutive elements (64 bytes of FP32 or 32 of BF16) of a row; four
-// rows per step with the next step's loads in flight; the amax of a row is
-// three shuffles within its 8 lanes; each lane ends up with the scale of one
-// of the 32 rows, so a block column of scales is one coalesced 128-byte store.
+// rows per step, a lane's loads of all its 8 rows (BF16) or of the next one
+// (FP32) in flight; the amax of a row is three shuffles within its 8 lanes;
+// each lane ends up with the scale of one of the 32 rows, so a block column
+// of scales is one coalesced 128-byte store.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -39,16 +40,30 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
     return r;
 }
 
-// 16 consecutive elements of a row as FP32.
+// 16 consecutive elements of a row: RAW 16-byte words (BF16: 2, FP32: 4)
 template <bool BF16_IN>
-__device__ __forceinline__ void load16(const void *x, long off, float (&v)[16])
+struct Raw16 {
+    static constexpr int WORDS = BF16_IN ? 2 : 4;
+    uint4 w[WORDS];
+};
+
+template <bool BF16_IN>
+__device__ __forceinline__ void load_raw16(const void *x, long off, Raw16<BF16_IN> &r)
+{
+    const uint4 *p = BF16_IN ? reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + off)
+                             : reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + off);
+#pragma unroll
+    for (int h = 0; h < Raw16<BF16_IN>::WORDS; ++h)
+        r.w[h] = __ldg(p + h);
+}
+
+template <bool BF16_IN>
+__device__ __forceinline__ void unpack16(const Raw16<BF16_IN> &r, float (&v)[16])
 {
     if constexpr (BF16_IN) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + off);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint4 raw = __ldg(p + h);
-            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            const uint32_t w[4] = {r.w[h].x, r.w[h].y, r.w[h].z, r.w[h].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 // a BF16 value is the high half of the FP32 with the same bits
@@ -57,14 +72,12 @@ __device__ __forceinline__ void load16(const void *x, long off, float (&v)[16])
             }
         }
     } else {
-        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + off);
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-            const float4 f = __ldg(p + h);
-            v[4 * h] = f.x;
-            v[4 * h + 1] = f.y;
-            v[4 * h + 2] = f.z;
-            v[4 * h + 3] = f.w;
+            v[4 * h] = __uint_as_float(r.w[h].x);
+            v[4 * h + 1] = __uint_as_float(r.w[h].y);
+            v[4 * h + 2] = __uint_as_float(r.w[h].z);
+            v[4 * h + 3] = __uint_as_float(r.w[h].w);
         }
     }
 }
@@ -96,22 +109,30 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32)
     const int sub = lane >> 3;                      // row within a step of 4
     const long col = (long)kb * 128 + (lane & 7) * 16;
     float my_scale = 0.0f;
-    float v[2][16];
-    auto load_step = [&](int it, float (&dst)[16]) {
+    // the lane's rows of the block in flight at once: all 8 for BF16 (64
+    // registers of raw data), 2 for FP32 (the next one loaded as the current
+    // one is consumed; more would lower the occupancy, measured slower)
+    constexpr int DEPTH = BF16_IN ? 8 : 2;
+    Raw16<BF16_IN> raw[DEPTH];
+    auto load_step = [&](int it, Raw16<BF16_IN> &dst) {
         const int row = r0 + it * 4 + sub;
-        if (row < M)
-            load16<BF16_IN>(x, (long)row * K + col, dst);
-        else
+        if (row < M) {
+            load_raw16<BF16_IN>(x, (long)row * K + col, dst);
+        } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                dst[e] = 0.0f;
+            for (int h = 0; h < Raw16<BF16_IN>::WORDS; ++h)
+                dst.w[h] = make_uint4(0u, 0u, 0u, 0u);
+        }
     };
-    load_step(0, v[0]);
+#pragma unroll
+    for (int it = 0; it < DEPTH; ++it)
+        load_step(it, raw[it]);
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
-        float(&w)[16] = v[it & 1];
-        if (it + 1 < 8)
-            load_step(it + 1, v[(it + 1) & 1]);
+        float w[16];
+        unpack16<BF16_IN>(raw[it % DEPTH], w);
+        if (it + DEPTH < 8)
+            load_step(it + DEPTH, raw[it % DEPTH]);
         float amax = 0.0f;
 #pragma unroll
         for (int e = 0; e < 16; ++e)

@@ -184,12 +184,19 @@ typedef struct dg_config {
     int cta_pair;   /* 2: a cluster of two CTAs computes each 256-row tile with
                        tcgen05 cta_group::2 MMAs (each CTA loads its own 128 rows
                        of A and half of the B tile); 1: one CTA per tile */
-    int swap_ab;    /* 1: the small-M dense kernel (M <= 128): each tile is
-                       128 rows of B (block_n = 128 columns of D) against all
-                       rows of A zero-padded to block_m, computed as D^T with
-                       B in the MMA's 128-row slot; split CTAs of a cluster
-                       share the tile's K range and reduce through distributed
-                       shared memory.  0: the kernels described above. */
+    int swap_ab;    /* 1: the small-M dense kernel (M <= 256): each tile is
+                       128 rows of B (block_n = 128 columns of D) against up to
+                       block_m rows of A (zero-padded; M > 128 in blocks of 128
+                       rows), computed as D^T with B in the MMA's 128-row slot;
+                       split CTAs of a cluster share the tile's K range and
+                       reduce through distributed shared memory.  0: the
+                       kernels described above. */
+    int tail_tiles; /* dense calls on the kernels above: tiles of the last,
+                       partly filled wave that form one block of D (the last
+                       M block from a 128-column boundary on) and are computed
+                       by the small-M kernel after the main kernel, which then
+                       runs whole waves (num_tiles - tail_tiles tiles); 0 =
+                       none */
 } dg_config;
 
 enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2, DG_KIND_DENSE_PER_TENSOR = 3 };
@@ -215,10 +222,16 @@ int dg_select_config(int kind, int M, int N, int K, int num_groups, int expected
  * shape is built, the split is outside 0..8, or cta_pair is not 0, 1 or 2. */
 int dg_force_config(int block_m, int block_n, int split, int cta_pair);
 
-/* Test hook: 0 = automatic (dense calls with M <= 128 use the small-M kernel
+/* Test hook: 0 = automatic (dense calls with M <= 256 use the small-M kernel
  * of dg_config.swap_ab), 1 = never use it, 2 = use it wherever it applies.
  * Returns DG_OK, or DG_ERR_INVALID_ARGUMENT for another mode. */
 int dg_force_swap_ab(int mode);
+
+/* Test hook for the split of a dense call's last partial wave
+ * (dg_config.tail_tiles): 0 = automatic (taken where the block layout allows
+ * it and the estimate says it is faster), 1 = never, 2 = wherever the layout
+ * allows it.  Returns DG_OK, or DG_ERR_INVALID_ARGUMENT for another mode. */
+int dg_force_tail_split(int mode);
 
 #ifdef __cplusplus
 }

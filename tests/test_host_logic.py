@@ -95,14 +95,22 @@ def test_block_n_example_tile_counts(lib):
 
 
 def test_selector_one_wave_for_small_prefill(lib):
-    """M=256, N=7168, K=2048 fits in one wave of 128-row tiles for every
-    BLOCK_N >= 112; measured on B200 the time per K block is flat in BLOCK_N
-    there, so the selector keeps one wave and a non-power-of-two width."""
-    for sms in (132, 148):
-        cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=sms)
-        assert cfg["block_m"] == 128 and cfg["split"] == 1
-        assert cfg["num_tiles"] <= sms and cfg["block_n"] >= 112
-        assert cfg["block_n"] & (cfg["block_n"] - 1) != 0
+    """M=256, N=7168, K=2048 (the README's SM-fill example).  The 128-row
+    kernels keep one wave of 128-row tiles with a non-power-of-two BLOCK_N
+    (measured on B200, the time per K block is flat in BLOCK_N there); by
+    default the small-M kernel takes the call: 2 x 56 tiles of 128 columns of
+    D, one wave of 112 CTAs."""
+    try:
+        fp8.force_swap_ab(1)
+        for sms in (132, 148):
+            cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=sms)
+            assert cfg["block_m"] == 128 and cfg["split"] == 1 and cfg["swap_ab"] == 0
+            assert cfg["num_tiles"] <= sms and cfg["block_n"] >= 112
+            assert cfg["block_n"] & (cfg["block_n"] - 1) != 0
+    finally:
+        fp8.force_swap_ab(0)
+    cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=148)
+    assert cfg["swap_ab"] == 1 and cfg["num_tiles"] == 112 and cfg["grid"] <= 148
 
 
 def test_selector_prefers_wide_tiles_for_large_shapes(lib):
@@ -121,7 +129,8 @@ def test_selector_prefers_wide_tiles_for_large_shapes(lib):
 
 def test_selector_invariants_and_determinism(lib):
     shapes = [(fp8.KIND_DENSE, m, n, k, 1, 0)
-              for m in (1, 64, 128, 300, 4096) for n in (8, 16, 2112, 7168) for k in (128, 7168)]
+              for m in (1, 64, 128, 200, 256, 300, 4096) for n in (8, 16, 2112, 7168)
+              for k in (128, 7168)]
     shapes += [(fp8.KIND_CONTIGUOUS, 128 * 40, 4096, 7168, 8, 0),
                (fp8.KIND_MASKED, 256, 4096, 7168, 16, 0),
                (fp8.KIND_MASKED, 256, 7168, 2048, 16, 100),
@@ -131,11 +140,14 @@ def test_selector_invariants_and_determinism(lib):
         b = fp8.select_config(kind, M, N, K, G, em, 148)
         assert a == b
         if a["swap_ab"]:
-            # small-M kernel: dense, M <= 128, tiles of 128 columns of D
-            assert kind == fp8.KIND_DENSE and M <= 128
-            assert a["block_m"] in (16, 32, 64, 128) and a["block_m"] >= M
+            # small-M kernel: dense, M <= 256, tiles of 128 columns of D by
+            # blocks of block_m rows
+            assert kind == fp8.KIND_DENSE and M <= 256
+            assert a["block_m"] in (16, 32, 64, 128)
+            assert a["block_m"] >= M or a["block_m"] == 128
             assert a["block_m"] // 2 < M or a["block_m"] == 16
-            assert a["block_n"] == 128 and a["num_tiles"] == -(-N // 128)
+            assert a["block_n"] == 128
+            assert a["num_tiles"] == -(-N // 128) * -(-M // a["block_m"])
             assert 1 <= a["split"] <= min(8, K // 128)
             assert a["grid"] % a["split"] == 0 and 1 <= a["grid"] <= 148
             assert a["stages"] >= min(2, K // 128) and a["smem_bytes"] <= 232448
@@ -197,8 +209,8 @@ def test_force_swap_ab(lib):
         fp8.force_swap_ab(2)
         fp8.force_config(128, 64)
         assert fp8.select_config(fp8.KIND_DENSE, 64, 2112, 7168, num_sms=148)["swap_ab"] == 1
-        # never for M > 128 or the grouped forms
-        assert fp8.select_config(fp8.KIND_DENSE, 129, 2112, 7168, num_sms=148)["swap_ab"] == 0
+        # never for M > 256 or the grouped forms
+        assert fp8.select_config(fp8.KIND_DENSE, 257, 2112, 7168, num_sms=148)["swap_ab"] == 0
         assert fp8.select_config(fp8.KIND_MASKED, 64, 4096, 7168, 4, 32, 148)["swap_ab"] == 0
         with pytest.raises(fp8.Fp8NtError):
             fp8.force_swap_ab(3)
@@ -210,13 +222,65 @@ def test_force_swap_ab(lib):
 def test_small_m_kernel_choice(lib):
     """MN is the smallest built width >= M; split never exceeds the K blocks;
     a lowered SM bound caps the clusters launched."""
-    for M, mn in ((1, 16), (16, 16), (17, 32), (33, 64), (64, 64), (65, 128), (128, 128)):
+    for M, mn in ((1, 16), (16, 16), (17, 32), (33, 64), (64, 64), (65, 128), (128, 128),
+                  (129, 128), (256, 128)):
         cfg = fp8.select_config(fp8.KIND_DENSE, M, 4096, 7168, num_sms=148)
         assert (cfg["swap_ab"], cfg["block_m"]) == (1, mn)
+    # 256 x 7168 x 2048 (the pages' SM-fill example shape): two 128-row blocks
+    # of A per 128 columns of D, 112 tiles on 112 SMs, the whole K on each
+    cfg = fp8.select_config(fp8.KIND_DENSE, 256, 7168, 2048, num_sms=148)
+    assert (cfg["num_tiles"], cfg["split"], cfg["grid"]) == (112, 1, 112)
     cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 256, num_sms=148)
     assert cfg["split"] <= 2
     cfg = fp8.select_config(fp8.KIND_DENSE, 64, 65536, 7168, num_sms=16)
     assert cfg["grid"] <= 16 and cfg["num_tiles"] == 512
+
+
+def test_tail_split_selection(lib):
+    """A dense call's last partial wave moves to the small-M kernel when its
+    tiles form one block of D: the last M block from a 128-column boundary
+    on.  4096 x 7168 x 2048 on 148 SMs: 896 tiles of 128 x 256, 6 whole waves
+    (888 tiles) and the last 8 tiles (rows 3968.., columns 5120..)."""
+    cfg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
+    assert (cfg["block_m"], cfg["block_n"], cfg["num_tiles"], cfg["grid"]) == (128, 256, 896, 148)
+    assert cfg["tail_tiles"] == 8
+    try:
+        fp8.force_tail_split(1)
+        assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["tail_tiles"] == 0
+        fp8.force_tail_split(2)
+        fp8.force_config(128, 256)
+        # 3 x 3 tiles on 8 SMs: one tile left, at column 512 of the last M block
+        assert fp8.select_config(fp8.KIND_DENSE, 320, 768, 1024, num_sms=8)["tail_tiles"] == 1
+        # 3 x 5 tiles on 6 SMs: three tiles left, all in the last M block
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 1280, 640, num_sms=6)["tail_tiles"] == 3
+        # 3 x 5 tiles on 4 SMs: 12 in whole waves, the last wave's 3 tiles are
+        # in the last M block; on 7 SMs (14 + 1) too; on 5 SMs the grid divides
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 1280, 640, num_sms=4)["tail_tiles"] == 3
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 1280, 640, num_sms=7)["tail_tiles"] == 1
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 1280, 640, num_sms=5)["tail_tiles"] == 0
+        # the partial wave spans two M blocks (4 x 5 tiles on 7 SMs: 14 + 6)
+        assert fp8.select_config(fp8.KIND_DENSE, 500, 1280, 640, num_sms=7)["tail_tiles"] == 0
+        # BLOCK_N = 192: the first tail column must be a multiple of 128
+        fp8.force_config(128, 192)
+        # (3 x 5 tiles: on 11 SMs the last 4 start at column 192, on 13 the
+        # last 2 at column 576: no; on 4 SMs the last 3 at column 384: yes)
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 960, 640, num_sms=11)["tail_tiles"] == 0
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 960, 640, num_sms=13)["tail_tiles"] == 0
+        assert fp8.select_config(fp8.KIND_DENSE, 300, 960, 640, num_sms=4)["tail_tiles"] == 3
+        # 256-row tiles: the last block's rows (at most 256) go to the small-M kernel
+        fp8.force_config(256, 128)
+        assert fp8.select_config(fp8.KIND_DENSE, 600, 640, 512, num_sms=4)["tail_tiles"] == 3
+        # never for the grouped forms, split-K, CTA pairs or per-tensor scales
+        fp8.force_config(0, 0)
+        assert fp8.select_config(fp8.KIND_MASKED, 256, 7168, 2048, 16, 128, 148)["tail_tiles"] == 0
+        assert fp8.select_config(fp8.KIND_DENSE_PER_TENSOR, 4096, 7168, 2048, num_sms=148)["tail_tiles"] == 0
+        fp8.force_config(256, 256, 0, 2)
+        assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["tail_tiles"] == 0
+        with pytest.raises(fp8.Fp8NtError):
+            fp8.force_tail_split(3)
+    finally:
+        fp8.force_tail_split(0)
+        fp8.force_config(0, 0)
 
 
 def test_force_config_rejects_unbuilt_shapes(lib):

@@ -1,7 +1,8 @@
-"""GPU parity of the small-M dense kernel (dense calls with M <= 128: tiles of
-128 columns of D computed transposed, the K range of a tile split over the
-CTAs of a cluster and reduced through distributed shared memory) against the
-CPU oracle, element by element, through the Python binding and the C ABI.
+"""GPU parity of the small-M dense kernel (dense calls with M <= 256: tiles of
+128 columns of D by blocks of up to 128 rows, computed transposed, the K range
+of a tile split over the CTAs of a cluster and combined through distributed
+shared memory) against the CPU oracle, element by element, through the Python
+binding and the C ABI.
 
 Covers every built width (MN = 16, 32, 64, 128) with M at and around its
 edges, every cluster size 1..8 (including more CTAs than K blocks), reuse of
@@ -61,6 +62,25 @@ def test_small_m_every_width(M):
     plus 8 columns), 5 K blocks."""
     prob = inputs.make_dense(M, 392, 640, seed=500 + M)
     run_and_compare(prob, f"small-M M={M}")
+
+
+@pytest.mark.parametrize("M", [129, 136, 200, 255, 256])
+def test_small_m_blocks_of_rows(M):
+    """M in (128, 256]: the kernel walks M in blocks of 128 rows (the last
+    one partial), each block its own tile; ragged N, 9 K blocks."""
+    prob = inputs.make_dense(M, 392, 128 * 9, seed=450 + M)
+    run_and_compare(prob, f"small-M blocks M={M}")
+
+
+@pytest.mark.parametrize("split", [1, 3, 8])
+def test_small_m_blocks_of_rows_split(split):
+    """Blocks of rows together with split K over a cluster."""
+    prob = inputs.make_dense(200, 264, 128 * 11, seed=470 + split)
+    fp8.force_config(0, 0, split)
+    try:
+        run_and_compare(prob, f"small-M blocks split={split}")
+    finally:
+        fp8.force_config(0, 0, 0)
 
 
 @pytest.mark.parametrize("split", [1, 2, 3, 4, 5, 6, 7, 8])
@@ -142,7 +162,8 @@ def test_small_m_no_stray_writes():
     assert not H.untouched(big[: prob.M]).any()
 
 
-@pytest.mark.parametrize("name", ["dense_decode_64x2112x7168", "dense_128x128x512"])
+@pytest.mark.parametrize("name", ["dense_decode_64x2112x7168", "dense_128x128x512",
+                                  "dense_prefill_256x7168x2048"])
 def test_small_m_full_size_all_elements(name):
     """The decode-shaped and 128x128x512 workloads, in the configuration the
     benchmark launches, every element against the oracle."""
