@@ -310,6 +310,6 @@ def force_swap_ab(mode: int = 0) -> None:
 
 def force_tail_split(mode: int = 0) -> None:
     """Split of a dense call's last partial wave onto the small-M kernel:
-    0 = automatic, 1 = never, 2 = wherever the block layout allows it.  For
-    tests."""
+    0 = automatic (off), 1 = never, 2 = wherever the block layout allows it,
+    3 = where the layout allows it and the cycle estimate favours it."""
     _check(load_library().dg_force_tail_split(int(mode)), "dg_force_tail_split")

@@ -98,9 +98,9 @@ std::atomic<int> g_num_sms_limit{0};
 std::atomic<uint32_t> g_forced{0};
 
 // swap: 0 = automatic, 1 = never the small-M (swap-AB) kernel, 2 = always
-// where it applies (dense calls with M <= 256).  tail: 0 = automatic, 1 =
-// never move a dense call's last partial wave to the small-M kernel, 2 =
-// wherever the layout allows it.
+// where it applies (dense calls with M <= 256).  tail: 0 = automatic (off),
+// 1 = never move a dense call's last partial wave to the small-M kernel, 2 =
+// wherever the layout allows it, 3 = where the estimate favours it.
 std::atomic<int> g_forced_swap{0};
 std::atomic<int> g_forced_tail{0};
 
@@ -718,8 +718,12 @@ int run_skinny(const Problem &pb, DeviceInfo *dev, int sms, const DenseView &v, 
 // last M block's rows (at most 256) by the remaining columns.  That block is
 // a small-M GEMM, which the small-M kernel spreads over the SMs with its K
 // range split over clusters; it runs after the main kernel, which then
-// computes whole waves only.  Taken when the small-M estimate (plus the gap
-// between two launches) is below the wave it replaces.
+// computes whole waves only.  Measured on B200 it is no faster than the
+// partial wave (dense 4096, 2048 and 8192 x 7168 x 2048: 81.2 / 50.9 / 143.3
+// us without, 81.6 / 50.7 / 145.4 us with: a wave of a few tiles alone runs
+// its K blocks faster than a full one), so it is taken only on request
+// (dg_force_tail_split), where the small-M estimate plus the gap between two
+// launches is below the wave it replaces or the request insists.
 struct TailSplit {
     int main_tiles; // tiles left to the main kernel
     int row0;       // the block's first row and column in D
@@ -733,7 +737,8 @@ bool plan_tail(const Problem &pb, const dg_config &cfg, int sms, int max_smem, D
                TailSplit *out)
 {
     const Forced f = forced_config();
-    if (pb.kind != DG_KIND_DENSE || cfg.split != 1 || cfg.cta_pair != 1 || cfg.swap_ab || f.tail == 1)
+    if (pb.kind != DG_KIND_DENSE || cfg.split != 1 || cfg.cta_pair != 1 || cfg.swap_ab || f.tail == 0 ||
+        f.tail == 1)
         return false;
     const long tiles = cfg.num_tiles, grid = cfg.grid;
     if (grid <= 0)
@@ -755,7 +760,7 @@ bool plan_tail(const Problem &pb, const dg_config &cfg, int sms, int max_smem, D
     SkinnyChoice ch;
     if (choose_skinny(sub, sms, max_smem, dev, &ch) != DG_OK)
         return false;
-    if (f.tail != 2) {
+    if (f.tail == 3) {
         double wave = 0;
         const int mw = cfg.block_m / 128;
         estimate_cycles(pb, mw, cfg.block_n, 1, 0, cfg.stages, sms, nullptr, &wave);
@@ -1140,7 +1145,7 @@ int dg_force_swap_ab(int mode)
 
 int dg_force_tail_split(int mode)
 {
-    if (mode < 0 || mode > 2)
+    if (mode < 0 || mode > 3)
         return DG_ERR_INVALID_ARGUMENT;
     g_forced_tail.store(mode, std::memory_order_relaxed);
     return DG_OK;

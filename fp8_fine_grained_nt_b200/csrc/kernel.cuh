@@ -75,13 +75,6 @@ struct KernelTraits {
     // buffers released together, which amortises the per-block handshake.
     static constexpr int GROUP_BY_REGS = PREFETCH ? 64 / COLS_PER_THREAD : 1;
     static constexpr int GROUP = GROUP_BY_REGS < NBUF / 2 ? GROUP_BY_REGS : (NBUF / 2 > 0 ? NBUF / 2 : 1);
-    // Wide tiles (two epilogue warpgroups, each owning BN / 2 columns of
-    // every row, read in two batches): each K block is issued as two MMAs of
-    // N = BN / 2, one per warpgroup's columns, each half with its own
-    // completion and release barriers, so that the MMAs into one half of a
-    // buffer wait only for the warpgroup that reads that half.
-    static constexpr bool HALVES = MW == 1 && !PAIR && !SCALAR && !PREFETCH;
-    static_assert(!HALVES || (BN / 2) % 16 == 0, "an M = 128 MMA takes N in multiples of 16");
     static constexpr uint32_t A_HALF_BYTES = HALF_M * BLOCK_K;
     static constexpr uint32_t B_BYTES = B_ROWS * BLOCK_K;
     static_assert(NBUF >= 2 && NBUF <= MAX_TMEM_BUFS && TMEM_NEED <= 512, "TMEM holds 512 columns");
@@ -367,12 +360,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t *sa_empty = sa_full + 2;
     uint64_t *mma_done = sa_empty + 2;
     uint64_t *tile_full = mma_done + 1; // per-tensor scaling: a tile's accumulator is complete (x2)
-    // split MMAs (T::HALVES): done_lo[j]: the first column half of K block
-    // j is complete (done[j] then covers the second half and frees the
-    // stage); tmem_empty[b] / tmem_empty_hi[b]: the first / second
-    // warpgroup has read its half of buffer b
-    uint64_t *done_lo = tile_full + 2;
-    uint64_t *tmem_empty_hi = done_lo + DONE_RING;
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + plan.off_misc);
     volatile uint32_t *abort_flag = misc + 1;
     int *prefix = reinterpret_cast<int *>(smem + plan.off_prefix);
@@ -387,15 +374,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int j = 0; j < DONE_RING; ++j)
             mbar_init(&done[j], 1);
         for (int b = 0; b < T::NBUF; ++b) {
-            // a pair's leader also counts the peer's epilogue warps; split
-            // MMAs: one warpgroup per half
-            mbar_init(&tmem_empty[b], PAIR ? 2 * NUM_EPI_WARPS : (T::HALVES ? 4 : NUM_EPI_WARPS));
-            if constexpr (T::HALVES)
-                mbar_init(&tmem_empty_hi[b], 4);
+            // a pair's leader also counts the peer's epilogue warps
+            mbar_init(&tmem_empty[b], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
         }
-        if constexpr (T::HALVES)
-            for (int j = 0; j < DONE_RING; ++j)
-                mbar_init(&done_lo[j], 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sb_full[b], 32);
             mbar_init(&sb_empty[b], NUM_EPI_WARPS);
@@ -625,40 +606,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     const uint64_t a_desc = a_desc0 + s * stage_step;
                     const uint64_t b_desc = b_desc0 + s * stage_step;
-                    if constexpr (T::HALVES) {
-                        // columns [0, BN/2) (B rows [0, BN/2)), then [BN/2, BN)
-                        // once the second warpgroup has read its half
-                        constexpr uint32_t idesc_h = make_idesc(BN / 2);
-                        const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS);
+                    for (int h = 0; h < halves; ++h) {
+                        const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS + h * BN);
 #pragma unroll
-                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
-                            mma_f8f6f4(d, a_desc + (uint64_t)((k * MMA_K) >> 4),
-                                       b_desc + (uint64_t)((k * MMA_K) >> 4), idesc_h, k > 0 ? 1u : 0u);
-                        mma_commit(&done_lo[kb_it % DONE_RING]);
-                        if (!wait_bar(&tmem_empty_hi[buf], ((kb_it / T::NBUF) & 1) ^ 1, abort_flag, p)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        // B rows from BN/2 on: BN/2 is a multiple of 8, so the
-                        // half starts on a 1024-byte swizzle atom
-                        const uint64_t b_hi = b_desc + (uint64_t)((BN / 2 * BLOCK_K) >> 4);
-#pragma unroll
-                        for (int k = 0; k < BLOCK_K / MMA_K; ++k)
-                            mma_f8f6f4(d + (uint32_t)(BN / 2), a_desc + (uint64_t)((k * MMA_K) >> 4),
-                                       b_hi + (uint64_t)((k * MMA_K) >> 4), idesc_h, k > 0 ? 1u : 0u);
-                    } else {
-                        for (int h = 0; h < halves; ++h) {
-                            const uint32_t d = tmem_base + (uint32_t)(buf * T::BUF_COLS + h * BN);
-#pragma unroll
-                            for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
-                                const uint64_t ad = a_desc + (uint64_t)((h * T::A_HALF_BYTES + k * MMA_K) >> 4);
-                                const uint64_t bd = b_desc + (uint64_t)((k * MMA_K) >> 4);
-                                if constexpr (PAIR)
-                                    mma_f8f6f4_pair(d, ad, bd, idesc, k > 0 ? 1u : 0u);
-                                else
-                                    mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
-                            }
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
+                            const uint64_t ad = a_desc + (uint64_t)((h * T::A_HALF_BYTES + k * MMA_K) >> 4);
+                            const uint64_t bd = b_desc + (uint64_t)((k * MMA_K) >> 4);
+                            if constexpr (PAIR)
+                                mma_f8f6f4_pair(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+                            else
+                                mma_f8f6f4(d, ad, bd, idesc, k > 0 ? 1u : 0u);
                         }
                     }
                     // one commit per K block frees its stage and publishes its
@@ -831,13 +788,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             auto buf_addr = [&](uint32_t it) {
                 return t_lane + (uint32_t)((int)(it % T::NBUF) * T::BUF_COLS);
             };
-            // split MMAs: the first warpgroup's half completes (and is
-            // released) on barriers of its own
-            uint64_t *const my_done = (T::HALVES && wg == 0) ? done_lo : done;
-            uint64_t *const my_empty = (T::HALVES && wg == 1) ? tmem_empty_hi : tmem_empty;
             // wait for K block `it`'s partial in TMEM
             auto wait_full = [&](uint32_t it) {
-                const bool r = wait_bar_warp(&my_done[it % DONE_RING], (it / DONE_RING) & 1, abort_flag, p);
+                const bool r = wait_bar_warp(&done[it % DONE_RING], (it / DONE_RING) & 1, abort_flag, p);
                 tc_fence_after();
                 return r;
             };
@@ -847,7 +800,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0)
                     for (int j = 0; j < cnt; ++j) {
-                        uint64_t *bar = &my_empty[(it + j) % T::NBUF];
+                        uint64_t *bar = &tmem_empty[(it + j) % T::NBUF];
                         if (PAIR && !leader)
                             mbar_arrive_cluster(map_shared_rank(smem_addr(bar), 0u));
                         else

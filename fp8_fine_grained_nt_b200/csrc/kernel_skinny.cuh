@@ -509,9 +509,11 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                 // has said so, every copy that read this CTA's partial tile
                 // has completed and the CTA may exit: the wait is left for
                 // the very end, after the sums, the stores and the TMEM
-                // release.
+                // release.  The barrier publishes no data (each copy's
+                // completion was observed on its owner's mbarrier before the
+                // owner arrives), so the arrive is relaxed.
                 __syncwarp();
-                cluster_arrive();
+                cluster_arrive_relaxed();
                 cluster_wait_pending = true;
             }
             const float *recv = reinterpret_cast<const float *>(smem + p.off_recv);

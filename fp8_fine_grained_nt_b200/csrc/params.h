@@ -111,9 +111,8 @@ __host__ __device__ inline SmemPlan make_smem_plan(int mw, int bn, int stages, i
     p.off_bars = align_up_u32(off, 8);
     // full per stage, the ring of "K block done" barriers, TMEM empty per
     // partial buffer, sb and sa full/empty x2, one "all MMAs done" barrier,
-    // two "tile accumulated" barriers (per-tensor scaling), and for MMAs
-    // split in column halves a second done ring and TMEM-empty set
-    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u + 2u + DONE_RING + MAX_TMEM_BUFS);
+    // two "tile accumulated" barriers (per-tensor scaling)
+    off = p.off_bars + 8u * (stages + DONE_RING + MAX_TMEM_BUFS + 8u + 1u + 2u);
     p.off_misc = align_up_u32(off, 16);
     p.total = p.off_misc + 16;
     return p;

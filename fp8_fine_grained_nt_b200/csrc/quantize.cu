@@ -14,11 +14,12 @@
 // full division.
 //
 // HBM-bound: one warp per 32 rows x 128 columns, 8 lanes per row, each lane
-// 16 consecutive elements (64 bytes of FP32 or 32 of BF16) of a row; four
-// rows per step, a lane's loads of all its 8 rows (BF16) or of the next one
-// (FP32) in flight; the amax of a row is three shuffles within its 8 lanes;
-// each lane ends up with the scale of one of the 32 rows, so a block column
-// of scales is one coalesced 128-byte store.
+// 16 elements of a row as 16-byte words (two of BF16, four of FP32): word h
+// of lane l is the row block's 16-byte word 8h + l, so that each load
+// instruction of a warp reads whole 128-byte lines; four rows per step, the
+// next rows' loads in flight; the amax of a row is three shuffles within its
+// 8 lanes; each lane ends up with the scale of one of the 32 rows, so a block
+// column of scales is one coalesced 128-byte store.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -47,14 +48,16 @@ struct Raw16 {
     uint4 w[WORDS];
 };
 
+// The lane's words of a row block starting at element `off`: word h is the
+// block's 16-byte word 8h + l8.
 template <bool BF16_IN>
-__device__ __forceinline__ void load_raw16(const void *x, long off, Raw16<BF16_IN> &r)
+__device__ __forceinline__ void load_raw16(const void *x, long off, int l8, Raw16<BF16_IN> &r)
 {
     const uint4 *p = BF16_IN ? reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + off)
                              : reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + off);
 #pragma unroll
     for (int h = 0; h < Raw16<BF16_IN>::WORDS; ++h)
-        r.w[h] = __ldg(p + h);
+        r.w[h] = __ldg(p + 8 * h + l8);
 }
 
 template <bool BF16_IN>
@@ -93,8 +96,17 @@ __device__ __forceinline__ float div_by_scale(float x, float s, float r)
     return e == 0.0f ? q0 : fmaf(e, r, q0);
 }
 
+// Rows in flight per lane and CTAs per SM asked of the compiler (so, the
+// registers each thread may use), measured on B200 (4096 x 7168): BF16 two
+// steps in flight at four CTAs per SM, FP32 four steps at one
 template <bool BF16_IN>
-__global__ void __launch_bounds__(QUANT_WARPS * 32)
+struct QuantShape {
+    static constexpr int DEPTH = BF16_IN ? 2 : 4;
+    static constexpr int MIN_CTAS = BF16_IN ? 4 : 1;
+};
+
+template <bool BF16_IN>
+__global__ void __launch_bounds__(QUANT_WARPS * 32, QuantShape<BF16_IN>::MIN_CTAS)
     quantize_1x128_kernel(const void *x, uint8_t *q, float *sa, int M, int K, long ld_sa)
 {
     const int lane = threadIdx.x & 31;
@@ -107,17 +119,15 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32)
     const int kb = (int)(wid % nkb);
     const int r0 = (int)(wid / nkb) * 32;
     const int sub = lane >> 3;                      // row within a step of 4
-    const long col = (long)kb * 128 + (lane & 7) * 16;
+    const int l8 = lane & 7;
+    const long col = (long)kb * 128;
     float my_scale = 0.0f;
-    // the lane's rows of the block in flight at once: all 8 for BF16 (64
-    // registers of raw data), 2 for FP32 (the next one loaded as the current
-    // one is consumed; more would lower the occupancy, measured slower)
-    constexpr int DEPTH = BF16_IN ? 8 : 2;
+    constexpr int DEPTH = QuantShape<BF16_IN>::DEPTH;
     Raw16<BF16_IN> raw[DEPTH];
     auto load_step = [&](int it, Raw16<BF16_IN> &dst) {
         const int row = r0 + it * 4 + sub;
         if (row < M) {
-            load_raw16<BF16_IN>(x, (long)row * K + col, dst);
+            load_raw16<BF16_IN>(x, (long)row * K + col, l8, dst);
         } else {
 #pragma unroll
             for (int h = 0; h < Raw16<BF16_IN>::WORDS; ++h)
@@ -152,9 +162,19 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32)
             packed[e / 4] = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
         }
         const int row = r0 + it * 4 + sub;
-        if (row < M)
-            *reinterpret_cast<uint4 *>(q + (long)row * K + col) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        if (row < M) {
+            // codes of word h: elements (8h + l8) * (16 / element size) on
+            uint8_t *dst = q + (long)row * K + col;
+            if constexpr (BF16_IN) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    *reinterpret_cast<uint2 *>(dst + (8 * h + l8) * 8) = make_uint2(packed[2 * h], packed[2 * h + 1]);
+            } else {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    *reinterpret_cast<uint32_t *>(dst + (8 * h + l8) * 4) = packed[h];
+            }
+        }
         // lane j keeps the scale of row j (rows it * 4 .. it * 4 + 3 now)
         const float sv = __shfl_sync(0xffffffffu, s, (lane & 3) * 8);
         if ((lane >> 2) == it)

@@ -191,12 +191,12 @@ typedef struct dg_config {
                        split CTAs of a cluster share the tile's K range and
                        reduce through distributed shared memory.  0: the
                        kernels described above. */
-    int tail_tiles; /* dense calls on the kernels above: tiles of the last,
-                       partly filled wave that form one block of D (the last
-                       M block from a 128-column boundary on) and are computed
-                       by the small-M kernel after the main kernel, which then
-                       runs whole waves (num_tiles - tail_tiles tiles); 0 =
-                       none */
+    int tail_tiles; /* dense calls on the kernels above, when requested with
+                       dg_force_tail_split: tiles of the last, partly filled
+                       wave that form one block of D (the last M block from a
+                       128-column boundary on) and are computed by the small-M
+                       kernel after the main kernel, which then runs whole
+                       waves (num_tiles - tail_tiles tiles); 0 = none */
 } dg_config;
 
 enum { DG_KIND_DENSE = 0, DG_KIND_CONTIGUOUS = 1, DG_KIND_MASKED = 2, DG_KIND_DENSE_PER_TENSOR = 3 };
@@ -227,10 +227,11 @@ int dg_force_config(int block_m, int block_n, int split, int cta_pair);
  * Returns DG_OK, or DG_ERR_INVALID_ARGUMENT for another mode. */
 int dg_force_swap_ab(int mode);
 
-/* Test hook for the split of a dense call's last partial wave
- * (dg_config.tail_tiles): 0 = automatic (taken where the block layout allows
- * it and the estimate says it is faster), 1 = never, 2 = wherever the layout
- * allows it.  Returns DG_OK, or DG_ERR_INVALID_ARGUMENT for another mode. */
+/* Opt-in split of a dense call's last partial wave (dg_config.tail_tiles):
+ * 0 = automatic, which is off (measured on B200 no faster than the partial
+ * wave), 1 = never, 2 = wherever the block layout allows it, 3 = where the
+ * block layout allows it and the cycle estimate favours it.  Returns DG_OK,
+ * or DG_ERR_INVALID_ARGUMENT for another mode. */
 int dg_force_tail_split(int mode);
 
 #ifdef __cplusplus

@@ -243,8 +243,10 @@ def test_tail_split_selection(lib):
     (888 tiles) and the last 8 tiles (rows 3968.., columns 5120..)."""
     cfg = fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)
     assert (cfg["block_m"], cfg["block_n"], cfg["num_tiles"], cfg["grid"]) == (128, 256, 896, 148)
-    assert cfg["tail_tiles"] == 8
+    assert cfg["tail_tiles"] == 0  # off unless requested (measured no faster)
     try:
+        fp8.force_tail_split(3)  # by the estimate
+        assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["tail_tiles"] == 8
         fp8.force_tail_split(1)
         assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["tail_tiles"] == 0
         fp8.force_tail_split(2)
@@ -277,7 +279,7 @@ def test_tail_split_selection(lib):
         fp8.force_config(256, 256, 0, 2)
         assert fp8.select_config(fp8.KIND_DENSE, 4096, 7168, 2048, num_sms=148)["tail_tiles"] == 0
         with pytest.raises(fp8.Fp8NtError):
-            fp8.force_tail_split(3)
+            fp8.force_tail_split(4)
     finally:
         fp8.force_tail_split(0)
         fp8.force_config(0, 0)

@@ -1,5 +1,5 @@
-"""GPU parity of the split of a dense call's last partial wave: the tiles of
-that wave that form one block of D (the last M block from a 128-column
+"""GPU parity of the opt-in split of a dense call's last partial wave: the
+tiles of that wave that form one block of D (the last M block from a 128-column
 boundary on) are computed by the small-M kernel after the main kernel, which
 runs whole waves only.  Every element is compared with the CPU oracle, with
 the split on and off, and the rows of D past M are checked untouched.
@@ -88,14 +88,18 @@ def test_tail_split_all_elements(M, N, K, bm, bn, sms, tail):
 
 
 def test_tail_split_full_size_block():
-    """Dense 4096 x 7168 x 2048 as the benchmark launches it: 888 tiles in
-    six whole waves and the last 8 (rows 3968.., columns 5120..) on the
-    small-M kernel.  The whole tail block, and the main kernel's rows and
+    """Dense 4096 x 7168 x 2048 with the split by estimate: 888 tiles in six
+    whole waves and the last 8 (rows 3968.., columns 5120..) on the small-M
+    kernel.  The whole tail block, and the main kernel's rows and
     columns next to it, against the oracle."""
     prob = inputs.make_workload("dense_prefill_4096x7168x2048")
-    cfg = fp8.select_config(fp8.KIND_DENSE, prob.M, prob.N, prob.K)
-    assert cfg["tail_tiles"] == 8
-    d = H.run_dense(prob)
+    fp8.force_tail_split(3)
+    try:
+        cfg = fp8.select_config(fp8.KIND_DENSE, prob.M, prob.N, prob.K)
+        assert cfg["tail_tiles"] == 8
+        d = H.run_dense(prob)
+    finally:
+        fp8.force_tail_split(0)
     check_status()
     got = H.bf16_bits_to_f64(d)
     r0, c0 = 3968, 5120
