@@ -414,15 +414,17 @@ def run_reference(args):
 
 # small calls timed as a batch in a CUDA graph: name -> number of distinct
 # problem sets the graph cycles through
-GRAPH_BATCHED = {"dense_decode_64x2112x7168": 16, "dense_128x128x512": 16}
+GRAPH_BATCHED = {"dense_decode_64x2112x7168": 16, "dense_128x128x512": 16,
+                 "dense_prefill_256x7168x2048": 16}
 
 
 def measure_graph_batched(fp8, name: str, rank: int, world: int, peaks, iters: int = 10) -> dict:
-    """Per-call device time of a decode-sized call, measured as a batch: one
-    CUDA graph holds `n` back-to-back calls, each on its own seeded problem
-    (distinct operands, as the layers of a model have distinct weights; for the
-    decode shape n x 15 MB of B exceeds the 126 MB L2, so every call reads its
-    weights from HBM), replayed `iters` times between CUDA events.  A single
+    """Per-call device time of a short call (decode-sized, or the 256-row
+    prefill), measured as a batch: one CUDA graph holds `n` back-to-back
+    calls, each on its own seeded problem (distinct operands, as the layers of
+    a model have distinct weights; for the decode shape n x 15 MB of B exceeds
+    the 126 MB L2, so every call reads its weights from HBM), replayed `iters`
+    times between CUDA events.  A single
     call timed between two events on this part carries several microseconds of
     launch and event overhead (an empty kernel reads ~5 us), which dominates a
     call whose roofline time is ~2.4 us; inside a graph only the gap between
