@@ -309,7 +309,7 @@ def oracle_sample(cases: list[Case], budget_s: float, seed: int = 0) -> dict:
     total_flops = sum(c.flops for c in cases)
     flops = 0.0
     elems = 0
-    batch = 64  # elements of the largest-FLOP workload per round, grown adaptively
+    batch = 64  # elements of the largest-FLOP workload per pass, grown adaptively
     start = time.time()
     while True:
         t0 = time.time()

@@ -11,7 +11,7 @@
 // step (Markstein's method: q0 = x * r, e = x - q0 * s exactly by FMA,
 // q = q0 + e * r), which yields the correctly rounded quotient when r is the
 // correctly rounded reciprocal, at three operations per element instead of a
-// full division.
+// full division, done on packed pairs of elements.
 //
 // HBM-bound: one warp per 32 rows x 128 columns, 8 lanes per row, each lane
 // 16 elements of a row as 16-byte words (two of BF16, four of FP32): word h
@@ -85,15 +85,32 @@ __device__ __forceinline__ void unpack16(const Raw16<BF16_IN> &r, float (&v)[16]
     }
 }
 
-// x / s rounded to nearest, given r = 1/s rounded to nearest: one FMA
-// correction of the product x * r (Markstein's method).  A zero residual
-// means q0 is exact; returning it keeps the sign of a zero quotient (-0 / s
-// is -0, which the correction q0 + 0 * r would turn into +0).
-__device__ __forceinline__ float div_by_scale(float x, float s, float r)
+// x / s rounded to nearest for two elements at once, given r = 1/s rounded
+// to nearest and ns = -s: one FMA correction of the product x * r
+// (Markstein's method: q0 = x r, e = x - q0 s exactly by FMA, q = q0 + e r),
+// on packed pairs (mul.rn / fma.rn .f32x2, rounded per element as the scalar
+// operations are).  s > 0, so the quotient has the sign of x; taking the sign
+// from x at the end keeps a zero quotient's sign (-0 / s is -0, which the
+// correction q0 + 0 * r would turn into +0) and changes nothing else.
+__device__ __forceinline__ void div2_by_scale(float x0, float x1, uint64_t r2, uint64_t ns2, float &y0,
+                                              float &y1)
 {
-    const float q0 = x * r;
-    const float e = fmaf(-q0, s, x);
-    return e == 0.0f ? q0 : fmaf(e, r, q0);
+    uint64_t x, q0, e, q;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(x), "l"(r2));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e) : "l"(q0), "l"(ns2), "l"(x));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(e), "l"(r2), "l"(q0));
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(q));
+    y0 = copysignf(a, x0);
+    y1 = copysignf(b, x1);
+}
+
+__device__ __forceinline__ uint64_t splat2(float v)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
 }
 
 // Rows in flight per lane and CTAs per SM asked of the compiler (so, the
@@ -151,14 +168,16 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32, QuantShape<BF16_IN>::MIN_CTA
         for (int d = 4; d > 0; d >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
         const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
-        const float r = __frcp_rn(s);
+        const uint64_t r2 = splat2(__frcp_rn(s)), ns2 = splat2(-s);
         uint32_t packed[4];
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
             float y[4];
+            div2_by_scale(w[e], w[e + 1], r2, ns2, y[0], y[1]);
+            div2_by_scale(w[e + 2], w[e + 3], r2, ns2, y[2], y[3]);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                y[i] = fminf(fmaxf(div_by_scale(w[e + i], s, r), -448.0f), 448.0f);
+                y[i] = fminf(fmaxf(y[i], -448.0f), 448.0f);
             packed[e / 4] = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
         }
         const int row = r0 + it * 4 + sub;
