@@ -404,7 +404,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC, "sample": "random output elements"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{elems} sampled output elements over all six workloads, "
+                         "sample": f"{elems} sampled output elements over all seven workloads, "
                                    f"proportional to FLOP, ~{budget:.0f}s per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -675,7 +675,7 @@ def run_gpu(args):
         r = oracle_sample(cases, args.cpu_budget_s)
         cpu = {"value": r["flops"] / r["seconds"] / 1e12, "unit": UNIT, "cores": r["cores"],
                "kind": "oracle",
-               "sample": f"{r['elements']} sampled output elements over all six workloads, "
+               "sample": f"{r['elements']} sampled output elements over all seven workloads, "
                          f"proportional to FLOP ({r['seconds']:.1f}s)"}
 
     if rank == 0:
