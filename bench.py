@@ -473,8 +473,9 @@ def measure_graph_batched(fp8, name: str, rank: int, world: int, peaks, iters: i
 def measure_next_rows(fp8, peaks, iters: int = 20) -> dict:
     """The rows built beyond the fine-grained GEMM, each timed alone (CUDA
     events around every call, L2 flushed before each): the 1x128 activation
-    quantiser, the per-tensor-scale GEMM and a skewed (Zipf-like) expert load
-    for the contiguous grouped GEMM."""
+    quantiser (also back to back over four inputs larger than the L2), the
+    per-tensor-scale GEMM and a skewed (Zipf-like) expert load for the
+    contiguous grouped GEMM."""
     dev = "cuda"
     flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -500,13 +501,29 @@ def measure_next_rows(fp8, peaks, iters: int = 20) -> dict:
     q = torch.empty(M, K, dtype=torch.uint8, device=dev)
     sa = torch.empty(K // 128, ld, dtype=torch.float32, device=dev)
     for name, dt, esz in (("fp32", torch.float32, 4), ("bf16", torch.bfloat16, 2)):
-        x = torch.randn(M, K, generator=g, device=dev).to(dt)
-        t = timed(lambda: fp8.quantize_fp8_1x128(x, q, sa))
+        # four distinct inputs (4 x 58 or 117 MB, above the L2) for the
+        # back-to-back timing below; the per-call timing uses the first
+        xs = [torch.randn(M, K, generator=g, device=dev).to(dt) for _ in range(4)]
+        t = timed(lambda: fp8.quantize_fp8_1x128(xs[0], q, sa))
         nbytes = esz * M * K + M * K + 4 * M * (K // 128)
-        out[f"quantize_1x128_{name}_{M}x{K}"] = {
-            "us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1), "bytes": nbytes,
-            "bound": "hbm", "roofline_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4)}
-        del x
+        row = {"us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1), "bytes": nbytes,
+               "bound": "hbm", "roofline_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4)}
+        # back to back: 20 calls cycling over the four inputs between one pair
+        # of events (each call's input was last read three calls earlier and
+        # has left the L2), so no per-call event or launch overhead is counted
+        for i in range(8):
+            fp8.quantize_fp8_1x128(xs[i % 4], q, sa)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(20):
+            fp8.quantize_fp8_1x128(xs[i % 4], q, sa)
+        e1.record(stream)
+        e1.synchronize()
+        tb = e0.elapsed_time(e1) * 1e-3 / 20
+        row["back_to_back"] = {"us": round(tb * 1e6, 2), "gbs": round(nbytes / tb / 1e9, 1),
+                               "roofline_frac": round(nbytes / tb / 1e9 / peaks["hbm_gbs"], 4)}
+        out[f"quantize_1x128_{name}_{M}x{K}"] = row
+        del xs
     M, N, K = 4096, 7168, 2048
     a = torch.randint(0, 0x7E, (M, K), generator=g, device=dev, dtype=torch.uint8)
     b = torch.randint(0, 0x7E, (N, K), generator=g, device=dev, dtype=torch.uint8)
