@@ -458,7 +458,11 @@ int cluster_capacity_model(int split, int sms)
 // block, (c) what one CTA's operand ring keeps in flight: measured on B200
 // (decode shape, 34 to 102 CTAs) a CTA takes in ~30 B/clk whatever the
 // number of CTAs, so more CTAs stream faster until (b) binds; plus set-up
-// and, with a cluster, the exchange of the partial tiles.
+// and, with a cluster, the exchange of the partial tiles (~4000 cycles and
+// more with the cluster's size: the partial tile's write, the bulk copies,
+// the wait for the slowest CTA, the sums, the closing barrier; traced at
+// ~4000-6000 cycles on the decode shape; 128x128x512 measured at 6.3 us per
+// call in a graph on one CTA against 7.3 us on a cluster of 2 or 4).
 double skinny_cycles(int M, int N, int K, int mn, int split, int cap)
 {
     const long tiles = (long)ceil_div(N, SKINNY_TILE_N) * ceil_div(M, mn);
@@ -471,7 +475,7 @@ double skinny_cycles(int M, int N, int K, int mn, int split, int cap)
     const double t_tma = (128.0 + mn) * 128.0 / 30.0;
     double t_kb = t_mma > t_hbm ? t_mma : t_hbm;
     t_kb = t_kb > t_tma ? t_kb : t_tma;
-    return (double)waves * (1200.0 + cnt * t_kb + (split > 1 ? 800.0 + 100.0 * split : 300.0));
+    return (double)waves * (1200.0 + cnt * t_kb + (split > 1 ? 4000.0 + 150.0 * split : 300.0));
 }
 
 struct SkinnyChoice {
