@@ -13,13 +13,13 @@
 // correctly rounded reciprocal, at three operations per element instead of a
 // full division, done on packed pairs of elements.
 //
-// HBM-bound: one warp per 32 rows x 128 columns, 8 lanes per row, each lane
-// 16 elements of a row as 16-byte words (two of BF16, four of FP32): word h
-// of lane l is the row block's 16-byte word 8h + l, so that each load
-// instruction of a warp reads whole 128-byte lines; four rows per step, the
-// next rows' loads in flight; the amax of a row is three shuffles within its
-// 8 lanes; each lane ends up with the scale of one of the 32 rows, so a block
-// column of scales is one coalesced 128-byte store.
+// HBM-bound: one warp per 32 (BF16) or 16 (FP32) rows x 128 columns, 8
+// lanes per row, each lane 16 elements of a row as 16-byte words (two of
+// BF16, four of FP32): word h of lane l is the row block's 16-byte word
+// 8h + l, so that each load instruction of a warp reads whole 128-byte lines;
+// four rows per step, the next rows' loads in flight; the amax of a row is
+// three shuffles within its 8 lanes; lane j ends up with the scale of the
+// warp's row j, so a block column of the warp's scales is one coalesced store.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -115,11 +115,14 @@ __device__ __forceinline__ uint64_t splat2(float v)
 
 // Rows in flight per lane and CTAs per SM asked of the compiler (so, the
 // registers each thread may use), measured on B200 (4096 x 7168): BF16 two
-// steps in flight at four CTAs per SM, FP32 four steps at one
+// steps in flight at four CTAs per SM, 32 rows per warp; FP32 four steps,
+// 16 rows per warp (its block column of scales is then 16 rows)
 template <bool BF16_IN>
 struct QuantShape {
-    static constexpr int DEPTH = BF16_IN ? 2 : 4;
+    static constexpr int ROWS = BF16_IN ? 32 : 16; // rows per warp, a multiple of 4, <= 32
+    static constexpr int DEPTH = BF16_IN ? 2 : 4;  // <= ROWS / 4
     static constexpr int MIN_CTAS = BF16_IN ? 4 : 1;
+    static_assert(ROWS % 4 == 0 && ROWS <= 32 && DEPTH >= 1 && DEPTH <= ROWS / 4, "row steps of 4 rows");
 };
 
 template <bool BF16_IN>
@@ -129,12 +132,13 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32, QuantShape<BF16_IN>::MIN_CTA
     const int lane = threadIdx.x & 31;
     const long wid = (long)blockIdx.x * QUANT_WARPS + (threadIdx.x >> 5);
     const int nkb = K / 128;
-    const long blocks = (long)((M + 31) / 32) * nkb;
+    constexpr int ROWS = QuantShape<BF16_IN>::ROWS;
+    const long blocks = (long)((M + ROWS - 1) / ROWS) * nkb;
     if (wid >= blocks)
         return;
-    // consecutive warps take consecutive K blocks of the same 32 rows
+    // consecutive warps take consecutive K blocks of the same ROWS rows
     const int kb = (int)(wid % nkb);
-    const int r0 = (int)(wid / nkb) * 32;
+    const int r0 = (int)(wid / nkb) * ROWS;
     const int sub = lane >> 3;                      // row within a step of 4
     const int l8 = lane & 7;
     const long col = (long)kb * 128;
@@ -155,10 +159,10 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32, QuantShape<BF16_IN>::MIN_CTA
     for (int it = 0; it < DEPTH; ++it)
         load_step(it, raw[it]);
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
+    for (int it = 0; it < ROWS / 4; ++it) {
         float w[16];
         unpack16<BF16_IN>(raw[it % DEPTH], w);
-        if (it + DEPTH < 8)
+        if (it + DEPTH < ROWS / 4)
             load_step(it + DEPTH, raw[it % DEPTH]);
         float amax = 0.0f;
 #pragma unroll
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32, QuantShape<BF16_IN>::MIN_CTA
         if ((lane >> 2) == it)
             my_scale = sv;
     }
-    if (r0 + lane < M)
+    if (lane < ROWS && r0 + lane < M)
         sa[(long)kb * ld_sa + r0 + lane] = my_scale;
 }
 
@@ -208,7 +212,8 @@ __global__ void __launch_bounds__(QUANT_WARPS * 32, QuantShape<BF16_IN>::MIN_CTA
 cudaError_t launch_quantize_1x128(const void *x, bool bf16_in, uint8_t *q, float *sa, int M, int K,
                                   long ld_sa, cudaStream_t stream)
 {
-    const long warps = (long)((M + 31) / 32) * (K / 128);
+    const int rows = bf16_in ? QuantShape<true>::ROWS : QuantShape<false>::ROWS;
+    const long warps = (long)((M + rows - 1) / rows) * (K / 128);
     const long grid = (warps + QUANT_WARPS - 1) / QUANT_WARPS;
     if (grid <= 0)
         return cudaSuccess;

@@ -232,6 +232,10 @@ def test_small_m_kernel_choice(lib):
     assert (cfg["num_tiles"], cfg["split"], cfg["grid"]) == (112, 1, 112)
     cfg = fp8.select_config(fp8.KIND_DENSE, 64, 2112, 256, num_sms=148)
     assert cfg["split"] <= 2
+    # 128x128x512 (four K blocks): one CTA, no cluster exchange (measured
+    # faster than a cluster of 2 or 4 on B200)
+    cfg = fp8.select_config(fp8.KIND_DENSE, 128, 128, 512, num_sms=148)
+    assert (cfg["swap_ab"], cfg["split"], cfg["grid"]) == (1, 1, 1)
     cfg = fp8.select_config(fp8.KIND_DENSE, 64, 65536, 7168, num_sms=16)
     assert cfg["grid"] <= 16 and cfg["num_tiles"] == 512
 
