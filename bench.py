@@ -61,6 +61,18 @@ WORKLOAD_NAMES = [
 WORKLOAD_DESC = ("dense 128x128x512 + decode 64x2112x7168 + prefill 4096x7168x2048 + "
                  "prefill 256x7168x2048 + contiguous 8 experts (4096,7168) + "
                  "masked 16x256 (4096,7168) + masked 16x256 (7168,2048), one call each per step")
+
+
+def bench_config(world: int) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": WORKLOAD_DESC,
+            "l2": "each step streams ~1.6 GB of distinct operands (> 126 MB L2); "
+                  "every call's operands are evicted by the rest of the step",
+            "parallelism": (f"{world} ranks, each an independent shard of every "
+                            "workload (dense: blocks of N; contiguous: experts; "
+                            "masked: groups)" if world > 1 else "1 GPU")}
+
+
 # launch-latency-bound: reported, not a roofline target
 LATENCY_BOUND = {"dense_128x128x512"}
 
@@ -401,8 +413,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "sample": "random output elements"},
+        "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": bench_config(args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{elems} sampled output elements over all seven workloads, "
                                    f"proportional to FLOP, ~{budget:.0f}s per step"},
@@ -701,12 +713,7 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "fp8_e4m3", "data": "synthetic",
-            "config": {"workload": WORKLOAD_DESC,
-                       "l2": "each step streams ~1.6 GB of distinct operands (> 126 MB L2); "
-                             "every call's operands are evicted by the rest of the step",
-                       "parallelism": (f"{world} ranks, each an independent shard of every "
-                                       "workload (dense: blocks of N; contiguous: experts; "
-                                       "masked: groups)" if world > 1 else "1 GPU")},
+            "config": bench_config(world),
             "per_shape": per_shape,
             "roofline": {"kernel": dom.name, "bound": bound, "achieved": round(achieved, 2),
                          "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
