@@ -523,13 +523,18 @@ __global__ void __launch_bounds__(SkinnyTraits<MN>::THREADS, 1)
                 const int n = n0 + c8;
                 if (n >= p.N)
                     continue;
+                // the slots' values summed in rank order (the loop unrolled
+                // over the largest cluster, so that the reads are issued ahead)
                 float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                for (int q = 0; q < p.split; ++q) {
-                    const float *src = recv + (size_t)q * (slot_bytes / 4) + (size_t)(it - lo) * 8;
-                    const float4 a = *reinterpret_cast<const float4 *>(src);
-                    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
-                    sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
-                    sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
+#pragma unroll
+                for (int q = 0; q < SKINNY_MAX_SPLIT; ++q) {
+                    if (q < p.split) {
+                        const float *src = recv + (size_t)q * (slot_bytes / 4) + (size_t)(it - lo) * 8;
+                        const float4 a = *reinterpret_cast<const float4 *>(src);
+                        const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+                        sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
+                        sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
+                    }
                 }
                 st_global_v4(p.D + (size_t)(m0 + m) * (size_t)p.ld_d + n, pack_bf16x2(sum[0], sum[1]),
                              pack_bf16x2(sum[2], sum[3]), pack_bf16x2(sum[4], sum[5]),
