@@ -184,3 +184,24 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
         steps, warmup, gpus, reference_budget_s = 1, 3, 2, 0.1
     assert bench.run_reference(A()) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    """Rank 0 of the reference arm (the CPU oracle on a bounded sample) prints
+    one JSON line with the same metric, unit, config and scaling as the
+    library's arm, plus its cpu_baseline and a zero-copy e2e."""
+    import json
+    import bench
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+
+    class A:
+        steps, warmup, gpus, reference_budget_s = 1, 1, 1, 0.2
+    assert bench.run_reference(A()) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["config"] == bench.bench_config(1) and line["scaling"] == "strong"
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
